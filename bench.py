@@ -1,0 +1,481 @@
+#!/usr/bin/env python3
+"""Benchmark of the gated Hyena long convolution on B200.
+
+Default workload: the long modal filter (hcl) over B=1, L=32768, D=4096, N=16
+real modes, bf16 x1/x2/x3 ~ N(0, 1), single pass.  One step = one call of
+hyena_modal_long_conv (coefficient synthesis + the scan kernel: every stage of
+the path, from loading x1/x2/x3 to storing y and the final state).
+
+Prints ONE JSON line (rank 0).  Metric: channel-tokens/s (one channel-token =
+one (b, t, c) output element); the roofline object reports the dominant
+kernel's achieved HBM bandwidth counted at 8 algorithmic bytes per
+channel-token (x1, x2, x3 read, y written, bf16 each) against the measured HBM
+peak.  Inputs (768 MB) are larger than L2 (126 MB), so no L2 flush is needed
+between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Multi-GPU (torchrun): the operator has no cross-GPU step on this path, so each
+rank runs an independent replica of the workload on its own GPU (weak
+scaling); ranks only meet for the barriers and the max-over-ranks timing.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "hcl long-conv channel-tokens/s at L=32K D=4096; achieved HBM GB/s vs peak"
+UNIT = "channel-tokens/s"
+BYTES_PER_CHTOK = 8  # 3 bf16 reads + 1 bf16 write
+
+WORKLOADS = {
+    "modal32k": dict(kind="modal", B=1, L=32768, D=4096, N=16, seed=2, chunk=None,
+                     desc="hcl modal long conv, B=1 L=32768 D=4096 N=16, single pass"),
+    "chunked131k": dict(kind="modal", B=1, L=131072, D=4096, N=16, seed=3, chunk=1024,
+                        desc="hcl modal long conv, B=1 L=131072 D=4096 N=16, 128 chunks of 1024 with carried state"),
+    "long262k": dict(kind="modal", B=1, L=262144, D=4096, N=16, seed=4, chunk=None, wide=True,
+                     desc="hcl modal long conv, B=1 L=262144 D=4096 N=16, wide dynamic range, single pass"),
+    "fir7": dict(kind="fir", B=2, L=8192, D=4096, K=7, seed=1,
+                 desc="hcs explicit FIR K=7, B=2 L=8192 D=4096"),
+    "fir128": dict(kind="fir", B=2, L=8192, D=4096, K=128, seed=1,
+                   desc="hcm explicit FIR K=128, B=2 L=8192 D=4096"),
+}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.5)  # let the sampler start before the timed region opens
+        except Exception:
+            self.proc = None
+        return self
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        import datetime
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        t0 = getattr(self, "start", None)
+        t1 = getattr(self, "end", None)
+        for line in getattr(self, "lines", []):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                ts = None
+            if ts is not None and t0 is not None and t1 is not None and not (t0 - 0.05 <= ts <= t1 + 0.05):
+                continue
+            try:
+                sm.append(float(parts[2]))
+                smax = float(parts[3])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[6:10]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle leg
+
+
+def oracle_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def oracle_sample_rate(wl, target_s=10.0):
+    """Times the fp64 oracle (as it stands) on a bounded sample of the workload.
+
+    The sample keeps all L tokens (so long-range decays are exercised) and a
+    subset of channels sized for roughly `target_s` seconds of CPU work.
+    Returns (channel-tokens/s, sample description, threads).
+    """
+    import oracle
+    from synth import make_fir_inputs, make_modal_inputs
+    threads = oracle_threads()
+    os.environ.setdefault("OMP_NUM_THREADS", str(threads))
+    L = wl["L"]
+    B = wl["B"]
+
+    def run(D):
+        if wl["kind"] == "modal":
+            inp = make_modal_inputs(B, L, D, wl["N"], wl["seed"], wl.get("wide", False))
+            t = time.perf_counter()
+            if wl.get("chunk"):
+                oracle.modal_chunked(inp["x1"], inp["x2"], inp["x3"], inp["log_poles"], inp["residues"],
+                                     inp["Dskip"], None, chunks=wl["chunk"])
+            else:
+                oracle.modal_recurrence(inp["x1"], inp["x2"], inp["x3"], inp["log_poles"],
+                                        inp["residues"], inp["Dskip"])
+            return time.perf_counter() - t
+        inp = make_fir_inputs(B, L, D, wl["K"], wl["seed"])
+        t = time.perf_counter()
+        oracle.fir(inp["x1"], inp["x2"], inp["x3"], inp["taps"], None, None)
+        return time.perf_counter() - t
+
+    oracle.build()
+    D0 = max(8, min(wl["D"], 8 * threads))
+    dt = run(D0)
+    rate = B * L * D0 / max(dt, 1e-9)
+    D1 = int(min(wl["D"], max(D0, rate * target_s / (B * L))))
+    D1 = max(8, D1 - D1 % 8)
+    if D1 > D0:
+        dt = run(D1)
+        rate = B * L * D1 / max(dt, 1e-9)
+    else:
+        D1 = D0
+    sample = f"B={B} L={L} D={D1} of {wl['D']} channels ({B * L * D1:.3g} channel-tokens), {dt:.1f} s"
+    return rate, sample, threads
+
+
+# ------------------------------------------------------------------ GPU leg
+
+
+def make_device_inputs(wl, device):
+    import torch
+    from synth import make_fir_inputs, make_modal_inputs
+
+    def up(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
+
+    if wl["kind"] == "modal":
+        inp = make_modal_inputs(wl["B"], wl["L"], wl["D"], wl["N"], wl["seed"], wl.get("wide", False))
+        host = dict(x1=inp["x1"], x2=inp["x2"], x3=inp["x3"])
+        dev = dict(x1=up(inp["x1"]), x2=up(inp["x2"]), x3=up(inp["x3"]),
+                   a=torch.from_numpy(inp["log_poles"]).to(device),
+                   R=torch.from_numpy(inp["residues"]).to(device),
+                   Ds=torch.from_numpy(inp["Dskip"]).to(device))
+        host.update(a=inp["log_poles"], R=inp["residues"], Ds=inp["Dskip"])
+    else:
+        inp = make_fir_inputs(wl["B"], wl["L"], wl["D"], wl["K"], wl["seed"])
+        host = dict(x1=inp["x1"], x2=inp["x2"], x3=inp["x3"], taps=inp["taps"])
+        dev = dict(x1=up(inp["x1"]), x2=up(inp["x2"]), x3=up(inp["x3"]), taps=up(inp["taps"]))
+    return host, dev
+
+
+class Step:
+    """One pass of the hot path over the resident inputs, via the C ABI."""
+
+    def __init__(self, wl, dev, device, graph=False):
+        import torch
+        import hyena_long_convolution_b200 as hy
+        self.hy = hy
+        self.wl = wl
+        self.dev = dev
+        B, L, D = wl["B"], wl["L"], wl["D"]
+        self.y = torch.empty((B, L, D), dtype=torch.bfloat16, device=device)
+        self.launches = 0
+        if wl["kind"] == "modal":
+            self.ws = hy.ModalWorkspace(B, D, wl["N"], device=device)
+            self.S = torch.zeros((B, D, wl["N"]), device=device)
+        self.graph = None
+        if graph:
+            s = torch.cuda.Stream(device=device)
+            s.wait_stream(torch.cuda.current_stream(device))
+            with torch.cuda.stream(s):
+                self._run()  # warm the per-device kernel attributes outside capture
+            torch.cuda.current_stream(device).wait_stream(s)
+            torch.cuda.synchronize(device)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self._run()
+            self.graph = g
+
+    def _run(self):
+        hy, wl, d = self.hy, self.wl, self.dev
+        n = 0
+        if wl["kind"] == "modal":
+            if wl.get("chunk"):
+                hy.modal_state_init(self.S)
+                n += hy.last_launch_count()
+                c = wl["chunk"]
+                for t0 in range(0, wl["L"], c):
+                    sl = slice(t0, t0 + c)
+                    hy.modal_long_conv(d["x1"][:, sl], d["x2"][:, sl], d["x3"][:, sl], d["a"], d["R"], d["Ds"],
+                                       y=self.y[:, sl], state_in=self.S, state_out=self.S, workspace=self.ws)
+                    n += hy.last_launch_count()
+            else:
+                hy.modal_long_conv(d["x1"], d["x2"], d["x3"], d["a"], d["R"], d["Ds"], y=self.y,
+                                   state_out=self.S, workspace=self.ws)
+                n += hy.last_launch_count()
+        else:
+            hy.short_conv(d["x1"], d["x2"], d["x3"], d["taps"], None, y=self.y)
+            n += hy.last_launch_count()
+        self.launches = n
+
+    def __call__(self):
+        if self.graph is not None:
+            self.graph.replay()
+        else:
+            self._run()
+
+
+def time_steps(step, steps, warmup, device):
+    import torch
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(device)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    stream = torch.cuda.current_stream(device)
+    for i in range(steps):
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(device)
+    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    return per
+
+
+def e2e_leg(wl, host, dev, device, steps, warmup):
+    """Same metric through the public binding with pinned host buffers: every
+    step copies x1/x2/x3 (and the filter parameters) host->device, runs the
+    operator and copies y device->host, all inside the timed region."""
+    import torch
+    import hyena_long_convolution_b200 as hy
+
+    def pin(a):
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if a.dtype == np.uint16 else a)
+        return t.pin_memory()
+
+    hx = {k: pin(v) for k, v in host.items()}
+    dx = {k: torch.empty(v.shape, dtype=v.dtype, device=device) for k, v in hx.items()}
+    y_host = torch.empty((wl["B"], wl["L"], wl["D"]), dtype=torch.int16).pin_memory()
+    B, L, D = wl["B"], wl["L"], wl["D"]
+    y = torch.empty((B, L, D), dtype=torch.bfloat16, device=device)
+    if wl["kind"] == "modal":
+        ws = hy.ModalWorkspace(B, D, wl["N"], device=device)
+
+    def step():
+        for k in hx:
+            dx[k].copy_(hx[k], non_blocking=True)
+        bf = {k: dx[k].view(torch.bfloat16) for k in ("x1", "x2", "x3")}
+        if wl["kind"] == "modal":
+            hy.modal_long_conv(bf["x1"], bf["x2"], bf["x3"], dx["a"], dx["R"], dx["Ds"], y=y, workspace=ws)
+        else:
+            hy.short_conv(bf["x1"], bf["x2"], bf["x3"], dx["taps"].view(torch.bfloat16), None, y=y)
+        y_host.copy_(y.view(torch.int16), non_blocking=True)
+
+    per = time_steps(step, steps, warmup, device)
+    h2d = sum(v.numel() * v.element_size() for v in hx.values())
+    d2h = y_host.numel() * y_host.element_size()
+    return per, h2d, d2h
+
+
+def run_gpu(args, wl):
+    import torch
+    world, rank, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+        pg = dist
+    import hyena_long_convolution_b200 as hy
+    hy.lib()  # fail loudly if the library is missing
+
+    host, dev = make_device_inputs(wl, device)
+    step = Step(wl, dev, device, graph=args.graph)
+    chtok = wl["B"] * wl["L"] * wl["D"]
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize(device)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    with ClockSampler(local) as clk:
+        clk.mark("start")
+        per = time_steps(step, args.steps, 0, device)
+        clk.mark("end")
+    barrier()
+    t_total_ms = sum(per)
+    ms_step = t_total_ms / args.steps
+    if pg is not None:
+        t = torch.tensor([t_total_ms], device=device)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        t_total_ms = float(t.item())
+        ms_step = t_total_ms / args.steps
+    value = world * chtok * args.steps / (t_total_ms / 1e3)
+
+    # e2e through the binding with host buffers (fewer steps: PCIe-bound)
+    e_steps = max(3, min(args.steps, 5))
+    eper, h2d, d2h = e2e_leg(wl, host, dev, device, e_steps, 3)
+    e_total = sum(eper)
+    if pg is not None:
+        t = torch.tensor([e_total], device=device)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e_total = float(t.item())
+    e_value = world * chtok * e_steps / (e_total / 1e3)
+
+    peak, peak_kind = measured_peaks()
+    per_sorted = sorted(per)
+    avg_ms = statistics.mean(per)
+    achieved = BYTES_PER_CHTOK * chtok / (avg_ms / 1e3) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        try:
+            with open(tpath) as f:
+                traffic = json.load(f).get(args.workload)
+        except Exception:
+            traffic = None
+
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "io_dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 inputs, pages' shapes)",
+        "config": {"workload": wl["desc"], "B": wl["B"], "L": wl["L"], "D": wl["D"],
+                   **({"N": wl["N"]} if wl["kind"] == "modal" else {"K": wl["K"]}),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "cache": "inputs larger than L2 (no flush)", "graph": bool(args.graph)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_kind} hbm_gbs (copy)",
+                     "algorithmic_bytes_per_launch": BYTES_PER_CHTOK * chtok,
+                     "kernel_ms_min": per_sorted[0], "kernel_ms_avg": avg_ms},
+        "e2e": {"value": e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e_total / e_steps},
+        "gpu_launches": step.launches * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, sample, threads = oracle_sample_rate(wl, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": sample}
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args, wl):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    rate_samples = []
+    sample = ""
+    threads = oracle_threads()
+    per_step = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup + args.steps):
+        rate, sample, threads = oracle_sample_rate(wl, per_step)
+        if i >= args.warmup:
+            rate_samples.append(rate)
+    value = statistics.mean(rate_samples)
+    chtok = wl["B"] * wl["L"] * wl["D"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": chtok / value * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl["desc"], "B": wl["B"], "L": wl["L"], "D": wl["D"]},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"per step: {sample}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="modal32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--graph", action="store_true", help="replay each step as a captured CUDA graph")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_gpu(args, wl)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,188 @@
+"""Gated Hyena cascade operator on NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI in include/hyena.h: every function below
+only checks and marshals torch tensors (device memory and streams) into raw
+pointers and sizes and calls the CUDA library; all arithmetic happens in the
+library's kernels.  There is no CPU path.
+
+    y = x3 * (h_c * (x1 * x2)) + Dskip * (x1 * x2)
+
+with h_c either an explicit short FIR (hcs 7 taps / hcm 128 taps,
+``short_conv``) or the long modal filter h_c[t] = sum_n R[c,n] exp(a[c,n] t)
+(hcl, ``modal_long_conv``).  Layout [B, L, D] bf16, channel-contiguous; a row
+stride ld >= D is allowed, so x1, x2, x3 may be views of one [B, L, 3D]
+projection output.
+"""
+from __future__ import annotations
+
+import ctypes
+
+from ._lib import HyenaError, check, lib  # noqa: F401
+
+__all__ = [
+    "HyenaError",
+    "ModalWorkspace",
+    "last_launch_count",
+    "modal_long_conv",
+    "modal_state_init",
+    "short_conv",
+    "workspace_check",
+    "workspace_size",
+]
+
+MAX_MODES = 16
+MAX_TAPS = 128
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _bld(x, name):
+    """[B, L, D] bf16 view with unit channel stride -> (B, L, D, ld)."""
+    torch = _torch()
+    if x.dtype != torch.bfloat16 or x.dim() != 3 or not x.is_cuda:
+        raise ValueError(f"{name} must be a 3-D bf16 CUDA tensor [B, L, D]")
+    B, L, D = x.shape
+    if x.stride(2) != 1:
+        raise ValueError(f"{name} must be channel-contiguous")
+    ld = x.stride(1) if L > 1 else (x.stride(0) // max(L, 1) if B > 1 else D)
+    if B > 1 and L > 0 and x.stride(0) != L * ld:
+        raise ValueError(f"{name}: batch stride must equal L * row stride")
+    return B, L, D, ld
+
+
+def _same_ld(*xs):
+    lds = {x[3] for x in xs}
+    if len(lds) != 1:
+        raise ValueError("x1, x2, x3 must share one row stride")
+
+
+def _f32(t, shape, name, allow_none=True):
+    torch = _torch()
+    if t is None:
+        if allow_none:
+            return None
+        raise ValueError(f"{name} is required")
+    if t.dtype != torch.float32 or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous fp32 tensor of shape {tuple(shape)}")
+    return t
+
+
+def last_launch_count() -> int:
+    """Kernels/memsets enqueued by the most recent call on this thread."""
+    return int(lib().hyena_last_launch_count())
+
+
+def workspace_size(B: int, D: int, N: int) -> int:
+    return int(lib().hyena_modal_long_conv_workspace_size(B, D, N))
+
+
+class ModalWorkspace:
+    """Device workspace for modal_long_conv, zero-filled once at creation."""
+
+    def __init__(self, B: int, D: int, N: int, device=None, stream=None):
+        torch = _torch()
+        n = workspace_size(B, D, N)
+        if n == 0:
+            raise ValueError("invalid workspace shape")
+        self.nbytes = n
+        self.buf = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+        check("hyena_modal_workspace_init",
+              lib().hyena_modal_workspace_init(_ptr(self.buf), n, _stream(stream)))
+
+    def fits(self, B: int, D: int, N: int) -> bool:
+        return workspace_size(B, D, N) <= self.nbytes
+
+
+def workspace_check(ws: ModalWorkspace, stream=None) -> None:
+    """Synchronise and raise if a bounded device wait of an earlier call ran out."""
+    check("hyena_workspace_check", lib().hyena_workspace_check(_ptr(ws.buf), _stream(stream)))
+
+
+def modal_state_init(state, stream=None):
+    """Zero a [B, D, N] fp32 modal state (start of chunked prefill)."""
+    B, D, N = state.shape
+    _f32(state, (B, D, N), "state", allow_none=False)
+    check("hyena_modal_state_init", lib().hyena_modal_state_init(_ptr(state), B, D, N, _stream(stream)))
+    return state
+
+
+def modal_long_conv(x1, x2, x3, log_poles, residues, Dskip=None, y=None, state_in=None,
+                    state_out=None, workspace: ModalWorkspace | None = None, stream=None):
+    """Long modal-form Hyena filter (hcl) with fused gates.
+
+    x1, x2, x3: [B, L, D] bf16 (views sharing a row stride); log_poles,
+    residues: [D, N] fp32; Dskip: [D] fp32 or None; state_in/state_out:
+    [B, D, N] fp32 or None (may be the same tensor).  Returns y ([B, L, D]
+    bf16, allocated if not given).
+    """
+    torch = _torch()
+    s1, s2, s3 = _bld(x1, "x1"), _bld(x2, "x2"), _bld(x3, "x3")
+    _same_ld(s1, s2, s3)
+    B, L, D, ld = s1
+    if s2[:3] != (B, L, D) or s3[:3] != (B, L, D):
+        raise ValueError("x1, x2, x3 shapes differ")
+    Dn, N = log_poles.shape
+    if Dn != D:
+        raise ValueError("log_poles must be [D, N]")
+    _f32(log_poles, (D, N), "log_poles", False)
+    _f32(residues, (D, N), "residues", False)
+    _f32(Dskip, (D,), "Dskip")
+    _f32(state_in, (B, D, N), "state_in")
+    _f32(state_out, (B, D, N), "state_out")
+    if y is None:
+        y = torch.empty((B, L, D), dtype=torch.bfloat16, device=x1.device)
+    yB, yL, yD, ld_y = _bld(y, "y")
+    if (yB, yL, yD) != (B, L, D):
+        raise ValueError("y shape differs from x")
+    if workspace is None:
+        workspace = ModalWorkspace(B, D, N, device=x1.device, stream=stream)
+    rc = lib().hyena_modal_long_conv(_ptr(x1), _ptr(x2), _ptr(x3), ld, _ptr(log_poles), _ptr(residues),
+                                     _ptr(Dskip), _ptr(y), ld_y, _ptr(state_in), _ptr(state_out),
+                                     B, L, D, N, _ptr(workspace.buf), workspace.nbytes, _stream(stream))
+    check("hyena_modal_long_conv", rc)
+    return y
+
+
+def short_conv(x1, x2, x3, taps, Dskip=None, y=None, hist_in=None, hist_out=None, stream=None):
+    """Explicit short Hyena FIR (hcs/hcm) with fused gates.
+
+    taps: [D, K] bf16 in lag order (taps[c, k] multiplies v[t-k]);
+    hist_in/hist_out: [B, K-1, D] fp32 or None (may be the same tensor).
+    """
+    torch = _torch()
+    s1, s2, s3 = _bld(x1, "x1"), _bld(x2, "x2"), _bld(x3, "x3")
+    _same_ld(s1, s2, s3)
+    B, L, D, ld = s1
+    if s2[:3] != (B, L, D) or s3[:3] != (B, L, D):
+        raise ValueError("x1, x2, x3 shapes differ")
+    if taps.dtype != torch.bfloat16 or taps.dim() != 2 or taps.shape[0] != D or not taps.is_contiguous():
+        raise ValueError("taps must be a contiguous bf16 [D, K] tensor")
+    K = taps.shape[1]
+    _f32(Dskip, (D,), "Dskip")
+    _f32(hist_in, (B, K - 1, D), "hist_in")
+    _f32(hist_out, (B, K - 1, D), "hist_out")
+    if y is None:
+        y = torch.empty((B, L, D), dtype=torch.bfloat16, device=x1.device)
+    yB, yL, yD, ld_y = _bld(y, "y")
+    if (yB, yL, yD) != (B, L, D):
+        raise ValueError("y shape differs from x")
+    rc = lib().hyena_short_conv(_ptr(x1), _ptr(x2), _ptr(x3), ld, _ptr(taps), _ptr(Dskip), _ptr(y), ld_y,
+                                _ptr(hist_in), _ptr(hist_out), B, L, D, K, _stream(stream))
+    check("hyena_short_conv", rc)
+    return y

@@ -1,0 +1,299 @@
+// api.cu -- the extern "C" entry points of libhyena_b200.so: argument checks,
+// TMA descriptor encoding, workspace layout and dispatch to the sm_100a
+// kernels.  Nothing here computes any part of the operator.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "hyena_internal.h"
+
+namespace hyena {
+
+namespace {
+
+thread_local int g_last_launches = 0;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+void resolve_encode()
+{
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 3-D bf16 tensor map over a [B, L, ld]-strided tensor, box [rows x 64 ch].
+bool encode_bf16_map(CUtensorMap *m, const void *base, int B, int L, int D, long long ld, int rows)
+{
+    std::call_once(g_encode_once, resolve_encode);
+    if (g_encode == nullptr) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
+                          static_cast<cuuint64_t>(B)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * 2,
+                             static_cast<cuuint64_t>(ld) * 2 * static_cast<cuuint64_t>(L)};
+    cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(rows), 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                                strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+hyena_status_t check_x(const void *x1, const void *x2, const void *x3, long long ld_x, const void *y,
+                       long long ld_y, int B, int L, int D)
+{
+    if (B < 1 || L < 0 || D < 1) return HYENA_ERR_INVALID_ARG;
+    if (L > 0) {
+        if (!x1 || !x2 || !x3 || !y) return HYENA_ERR_INVALID_ARG;
+        if (ld_x < D || ld_y < D) return HYENA_ERR_INVALID_ARG;
+        if ((ld_x % 8) || (ld_y % 8)) return HYENA_ERR_ALIGNMENT;
+        if (!aligned16(x1) || !aligned16(x2) || !aligned16(x3) || !aligned16(y))
+            return HYENA_ERR_ALIGNMENT;
+        // element offsets must fit the 32-bit TMA coordinates and 40-bit strides
+        if (static_cast<long long>(L) * ld_x * 2 >= (1ll << 40)) return HYENA_ERR_UNSUPPORTED;
+    }
+    if (D % 8) return HYENA_ERR_ALIGNMENT;
+    return HYENA_OK;
+}
+
+hyena_status_t copy_or_zero(float *dst, const float *src, size_t bytes, cudaStream_t st, int &launches)
+{
+    if (dst == nullptr) return HYENA_OK;
+    if (src == dst) return HYENA_OK;
+    const cudaError_t e = src ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st)
+                              : cudaMemsetAsync(dst, 0, bytes, st);
+    if (e != cudaSuccess) return HYENA_ERR_CUDA;
+    ++launches;
+    return HYENA_OK;
+}
+
+}  // namespace
+
+ModalLayout modal_layout(int B, int D, int N)
+{
+    ModalLayout L;
+    L.NP = modal_padded_modes(N);
+    L.nCB = (D + MCH - 1) / MCH;
+    L.Dp = L.nCB * MCH;
+    const size_t tab = static_cast<size_t>(L.NP) * L.Dp * sizeof(float);
+    size_t off = 0;
+    L.off_hdr = off;
+    off += 256;
+    L.off_cP = off;
+    off = align256(off + tab);
+    L.off_cR = off;
+    off = align256(off + tab);
+    L.off_cPw = off;
+    off = align256(off + tab * (MW + 1));
+    L.off_cDs = off;
+    off = align256(off + static_cast<size_t>(L.Dp) * sizeof(float));
+    const size_t chains = static_cast<size_t>(B) * L.nCB;
+    L.off_flags = off;
+    off = align256(off + chains * MRING * sizeof(unsigned long long));
+    L.off_slots = off;
+    off = align256(off + chains * MRING * 2 * L.NP * MCH * sizeof(float));
+    L.total = off;
+    return L;
+}
+
+}  // namespace hyena
+
+using namespace hyena;
+
+extern "C" {
+
+const char *hyena_status_string(hyena_status_t s)
+{
+    switch (s) {
+        case HYENA_OK: return "HYENA_OK";
+        case HYENA_ERR_INVALID_ARG: return "HYENA_ERR_INVALID_ARG";
+        case HYENA_ERR_ALIGNMENT: return "HYENA_ERR_ALIGNMENT";
+        case HYENA_ERR_UNSUPPORTED: return "HYENA_ERR_UNSUPPORTED";
+        case HYENA_ERR_CUDA: return "HYENA_ERR_CUDA";
+        case HYENA_ERR_TIMEOUT: return "HYENA_ERR_TIMEOUT";
+        case HYENA_ERR_WORKSPACE: return "HYENA_ERR_WORKSPACE";
+        default: return "HYENA_ERR_UNKNOWN";
+    }
+}
+
+int hyena_abi_version(void) { return 100; }
+
+int hyena_last_launch_count(void) { return g_last_launches; }
+
+hyena_status_t hyena_short_conv(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
+                                int64_t ld_x, const hyena_bf16_t *taps, const float *Dskip,
+                                hyena_bf16_t *y, int64_t ld_y, const float *hist_in, float *hist_out,
+                                int B, int L, int D, int K, void *stream)
+{
+    hyena_status_t st = check_x(x1, x2, x3, ld_x, y, ld_y, B, L, D);
+    if (st != HYENA_OK) return st;
+    if (K < 1 || K > HYENA_MAX_TAPS) return K < 1 ? HYENA_ERR_INVALID_ARG : HYENA_ERR_UNSUPPORTED;
+    if (taps == nullptr) return HYENA_ERR_INVALID_ARG;
+    if ((Dskip && !aligned16(Dskip)) || (hist_in && !aligned16(hist_in)) ||
+        (hist_out && !aligned16(hist_out)) || !aligned16(taps))
+        return HYENA_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int launches = 0;
+    if (L == 0) {
+        if (K > 1) {
+            st = copy_or_zero(hist_out, hist_in, static_cast<size_t>(B) * (K - 1) * D * sizeof(float), s,
+                              launches);
+            if (st != HYENA_OK) return st;
+        }
+        g_last_launches = launches;
+        return HYENA_OK;
+    }
+    FirArgs a{};
+    a.taps = taps;
+    a.Dskip = Dskip;
+    a.y = y;
+    a.ld_y = ld_y;
+    a.hist_in = hist_in;
+    a.B = B;
+    a.L = L;
+    a.D = D;
+    a.K = K;
+    a.HR = fir_halo_rows(K);
+    a.x1 = x1;
+    a.x2 = x2;
+    a.ld_x = ld_x;
+    a.hist_out = hist_out;
+    CUtensorMap m1, m2, m3, h1, h2;
+    if (!encode_bf16_map(&m1, x1, B, L, D, ld_x, FT) || !encode_bf16_map(&m2, x2, B, L, D, ld_x, FT) ||
+        !encode_bf16_map(&m3, x3, B, L, D, ld_x, FT))
+        return HYENA_ERR_CUDA;
+    if (a.HR > 0) {
+        if (!encode_bf16_map(&h1, x1, B, L, D, ld_x, a.HR) || !encode_bf16_map(&h2, x2, B, L, D, ld_x, a.HR))
+            return HYENA_ERR_CUDA;
+    } else {
+        h1 = m1;
+        h2 = m2;
+    }
+    const int n = launch_fir(m1, m2, m3, h1, h2, a, s);
+    if (n < 0) return HYENA_ERR_CUDA;
+    g_last_launches = n;
+    return HYENA_OK;
+}
+
+size_t hyena_modal_long_conv_workspace_size(int B, int D, int N)
+{
+    if (B < 1 || D < 1 || N < 1 || N > HYENA_MAX_MODES) return 0;
+    return modal_layout(B, D, N).total;
+}
+
+hyena_status_t hyena_modal_workspace_init(void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (workspace == nullptr || workspace_bytes == 0) return HYENA_ERR_INVALID_ARG;
+    if (cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return HYENA_ERR_CUDA;
+    g_last_launches = 1;
+    return HYENA_OK;
+}
+
+hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
+                                     int64_t ld_x, const float *log_poles, const float *residues,
+                                     const float *Dskip, hyena_bf16_t *y, int64_t ld_y,
+                                     const float *state_in, float *state_out, int B, int L, int D, int N,
+                                     void *workspace, size_t workspace_bytes, void *stream)
+{
+    hyena_status_t st = check_x(x1, x2, x3, ld_x, y, ld_y, B, L, D);
+    if (st != HYENA_OK) return st;
+    if (N < 1) return HYENA_ERR_INVALID_ARG;
+    if (N > HYENA_MAX_MODES) return HYENA_ERR_UNSUPPORTED;
+    if (!log_poles || !residues) return HYENA_ERR_INVALID_ARG;
+    if (!aligned16(log_poles) || !aligned16(residues) || (Dskip && !aligned16(Dskip)) ||
+        (state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
+        return HYENA_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int launches = 0;
+    if (L == 0) {
+        st = copy_or_zero(state_out, state_in, static_cast<size_t>(B) * D * N * sizeof(float), s, launches);
+        if (st != HYENA_OK) return st;
+        g_last_launches = launches;
+        return HYENA_OK;
+    }
+    const ModalLayout lay = modal_layout(B, D, N);
+    if (workspace == nullptr || workspace_bytes < lay.total) return HYENA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return HYENA_ERR_ALIGNMENT;
+    const long long nseg = (static_cast<long long>(L) + MT - 1) / MT;
+    const long long units = nseg * B * lay.nCB;
+    if (units >= (1ll << 31)) return HYENA_ERR_UNSUPPORTED;
+
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    ModalArgs a{};
+    a.y = y;
+    a.ld_y = ld_y;
+    a.state_in = state_in;
+    a.state_out = state_out;
+    a.B = B;
+    a.L = L;
+    a.D = D;
+    a.N = N;
+    a.nCB = lay.nCB;
+    a.Dp = lay.Dp;
+    a.nUnits = static_cast<unsigned int>(units);
+    a.cP = reinterpret_cast<const float *>(ws + lay.off_cP);
+    a.cR = reinterpret_cast<const float *>(ws + lay.off_cR);
+    a.cPw = reinterpret_cast<const float *>(ws + lay.off_cPw);
+    a.cDs = reinterpret_cast<const float *>(ws + lay.off_cDs);
+    a.flags = reinterpret_cast<unsigned long long *>(ws + lay.off_flags);
+    a.slots = reinterpret_cast<float *>(ws + lay.off_slots);
+    a.hdr = reinterpret_cast<unsigned int *>(ws + lay.off_hdr);
+
+    ModalSynthArgs sy{};
+    sy.log_poles = log_poles;
+    sy.residues = residues;
+    sy.Dskip = Dskip;
+    sy.D = D;
+    sy.N = N;
+    sy.Dp = lay.Dp;
+    sy.cP = reinterpret_cast<float *>(ws + lay.off_cP);
+    sy.cR = reinterpret_cast<float *>(ws + lay.off_cR);
+    sy.cPw = reinterpret_cast<float *>(ws + lay.off_cPw);
+    sy.cDs = reinterpret_cast<float *>(ws + lay.off_cDs);
+
+    CUtensorMap m1, m2, m3;
+    if (!encode_bf16_map(&m1, x1, B, L, D, ld_x, MT) || !encode_bf16_map(&m2, x2, B, L, D, ld_x, MT) ||
+        !encode_bf16_map(&m3, x3, B, L, D, ld_x, MT))
+        return HYENA_ERR_CUDA;
+    const int n = launch_modal(m1, m2, m3, a, sy, lay.NP, s);
+    if (n < 0) return HYENA_ERR_CUDA;
+    g_last_launches = n;
+    return HYENA_OK;
+}
+
+hyena_status_t hyena_modal_state_init(float *state, int B, int D, int N, void *stream)
+{
+    if (state == nullptr || B < 1 || D < 1 || N < 1) return HYENA_ERR_INVALID_ARG;
+    if (cudaMemsetAsync(state, 0, static_cast<size_t>(B) * D * N * sizeof(float),
+                        static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return HYENA_ERR_CUDA;
+    g_last_launches = 1;
+    return HYENA_OK;
+}
+
+hyena_status_t hyena_workspace_check(void *workspace, void *stream)
+{
+    if (workspace == nullptr) return HYENA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return HYENA_ERR_CUDA;
+    unsigned int err = 0;
+    unsigned int *hdr = static_cast<unsigned int *>(workspace);
+    if (cudaMemcpy(&err, hdr + 2, sizeof err, cudaMemcpyDeviceToHost) != cudaSuccess) return HYENA_ERR_CUDA;
+    if (err != 0u) {
+        if (cudaMemset(hdr + 2, 0, sizeof err) != cudaSuccess) return HYENA_ERR_CUDA;
+        return HYENA_ERR_TIMEOUT;
+    }
+    return HYENA_OK;
+}
+
+}  // extern "C"

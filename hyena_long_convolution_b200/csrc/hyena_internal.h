@@ -1,0 +1,87 @@
+// hyena_internal.h -- host-side declarations shared by the entry points and
+// the kernel launchers (not part of the public interface).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/hyena.h"
+
+namespace hyena {
+
+// ---------------------------------------------------------------- modal scan
+// Work unit: MCH channels x MT tokens of one batch row.  One CTA of MW warps
+// processes a unit; warp w owns tokens [w*MS, (w+1)*MS) of it and lane l the
+// channel pair (2l, 2l+1).
+constexpr int MCH = 64;
+constexpr int MT = 128;
+constexpr int MW = 8;
+constexpr int MS = MT / MW;
+constexpr int MRING = 32;  // ring slots per (batch row, channel block) chain
+constexpr int MLB = 16;    // deepest look-back, in units
+
+inline int modal_padded_modes(int N) { return N <= 4 ? 4 : (N <= 8 ? 8 : 16); }
+
+struct ModalLayout {
+    int NP = 0, nCB = 0, Dp = 0;
+    size_t off_hdr = 0, off_cP = 0, off_cR = 0, off_cPw = 0, off_cDs = 0, off_flags = 0,
+           off_slots = 0, total = 0;
+};
+
+ModalLayout modal_layout(int B, int D, int N);
+
+struct ModalArgs {
+    uint16_t *y;
+    long long ld_y;
+    const float *state_in;
+    float *state_out;
+    int B, L, D, N;
+    int nCB, Dp;
+    unsigned int nUnits;
+    const float *cP;    // [NP][Dp]  exp(a)
+    const float *cR;    // [NP][Dp]  residues
+    const float *cPw;   // [MW+1][NP][Dp]  exp(a * MS * w)
+    const float *cDs;   // [Dp]  skip
+    unsigned long long *flags;  // [B*nCB][MRING]
+    float *slots;       // [B*nCB][MRING][2][NP][MCH]
+    unsigned int *hdr;  // [0] ticket, [1] finished CTAs, [2] error bits, [3] epoch
+};
+
+struct ModalSynthArgs {
+    const float *log_poles, *residues, *Dskip;
+    int D, N, Dp;
+    float *cP, *cR, *cPw, *cDs;
+};
+
+// Launches the coefficient-synthesis kernel and the scan kernel; returns the
+// number of launches enqueued or a negative value on a CUDA error.
+int launch_modal(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3,
+                 const ModalArgs &a, const ModalSynthArgs &s, int NP, cudaStream_t st);
+
+// ---------------------------------------------------------------- short FIR
+constexpr int FCH = 64;   // channels per CTA
+constexpr int FT = 128;   // output tokens per CTA
+constexpr int FW = 8;     // warps per CTA
+constexpr int FRW = FT / FW;  // output rows per warp
+
+inline int fir_halo_rows(int K) { return K <= 1 ? 0 : ((K - 1 + 7) / 8) * 8; }
+
+struct FirArgs {
+    const uint16_t *taps;
+    const float *Dskip;
+    uint16_t *y;
+    long long ld_y;
+    const float *hist_in;
+    int B, L, D, K, HR;
+    const uint16_t *x1, *x2;  // for the history kernel
+    long long ld_x;
+    float *hist_out;
+};
+
+int launch_fir(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3,
+               const CUtensorMap &h1, const CUtensorMap &h2, const FirArgs &a,
+               cudaStream_t st);
+
+}  // namespace hyena

@@ -1,0 +1,238 @@
+// short_conv.cu -- explicit short causal FIR (hcs: 7 taps, hcm: 128 taps)
+// with the fused Hyena gates, on sm_100a.
+//
+// Operator (Evo2-7B-262K model card, §Implementation Notes: "Block dispatch"
+// names FIR cascades of inner length 7 and 128; "Custom cache" and the
+// Evo1-1.5-7B-8K card's "Cache subclass" carry the FIR window):
+//   v[t] = x1[t] x2[t];  conv[t] = sum_{k<K} taps[c,k] v[t-k];
+//   y[t] = x3[t] conv[t] + Dskip[c] v[t].
+//
+// Design.  One CTA owns FCH = 64 channels x FT = 128 output tokens of one
+// batch row.  TMA stages x1, x2 for the tile plus a halo of HR >= K-1 earlier
+// rows (a second, shorter box) and x3 for the tile; v = x1 x2 is formed once in
+// fp32 into shared memory (halo rows before t = 0 come from hist_in).  Warp w
+// computes FRW = 16 consecutive outputs for the lane's two channels with a
+// register-blocked sliding window: per block of 8 taps it loads the 8 taps and
+// the 23 window values it needs and issues 8 x 16 packed f32x2 FMAs.  The
+// gates are applied in registers and y is stored as coalesced 128-byte rows.
+// A second small kernel writes hist_out (the last K-1 values of v).
+#include "hyena_device.cuh"
+#include "hyena_internal.h"
+
+namespace hyena {
+
+namespace {
+
+constexpr int kMaxHalo = 128;  // HR <= 128 since K <= 128
+constexpr int kRowWords = FCH / 2;  // 32-bit words per bf16 row
+
+struct FirSmemView {
+    uint32_t *x1, *x2, *x3;  // [HR + FT][32], [HR + FT][32], [FT][32]
+    float2 *v;               // [HR + FT][32]
+    float2 *taps;            // [K][32]
+    uint64_t *bar;
+};
+
+__host__ __device__ inline size_t fir_smem_bytes(int HR, int K)
+{
+    const size_t rows = static_cast<size_t>(HR) + FT;
+    return rows * kRowWords * 4 * 2 + static_cast<size_t>(FT) * kRowWords * 4 + rows * 32 * 8 +
+           static_cast<size_t>(K) * 32 * 8 + 16;
+}
+
+__device__ inline FirSmemView fir_smem(unsigned char *base, int HR, int K)
+{
+    FirSmemView s;
+    const int rows = HR + FT;
+    s.x1 = reinterpret_cast<uint32_t *>(base);
+    s.x2 = s.x1 + rows * kRowWords;
+    s.x3 = s.x2 + rows * kRowWords;
+    s.v = reinterpret_cast<float2 *>(s.x3 + FT * kRowWords);
+    s.taps = s.v + rows * 32;
+    s.bar = reinterpret_cast<uint64_t *>(s.taps + K * 32);
+    return s;
+}
+
+// Accumulates taps [kb, kb + nq) into acc for this warp's FRW outputs.
+template <int NQ>
+__device__ __forceinline__ void fir_block(float2 (&acc)[FRW], const float2 *vbase,
+                                          const float2 *tbase, int lane)
+{
+    // vbase points at v row (first output row - kb - (NQ-1)), this lane.
+    float2 tq[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) tq[q] = tbase[q * 32 + lane];
+    float2 w[FRW + NQ - 1];
+#pragma unroll
+    for (int j = 0; j < FRW + NQ - 1; ++j) w[j] = vbase[j * 32 + lane];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+#pragma unroll
+        for (int i = 0; i < FRW; ++i) acc[i] = __ffma2_rn(tq[q], w[i - q + NQ - 1], acc[i]);
+}
+
+__global__ void __launch_bounds__(FW * 32)
+    fir_kernel(const __grid_constant__ CUtensorMap tm1, const __grid_constant__ CUtensorMap tm2,
+               const __grid_constant__ CUtensorMap tm3, const __grid_constant__ CUtensorMap th1,
+               const __grid_constant__ CUtensorMap th2, const FirArgs A)
+{
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const int HR = A.HR;
+    const int K = A.K;
+    FirSmemView sm = fir_smem(smem_raw, HR, K);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int cb = blockIdx.x;
+    const int t0 = blockIdx.y * FT;
+    const int b = blockIdx.z;
+    const int c0 = cb * FCH + 2 * lane;
+    const bool ch_ok = c0 < A.D;
+
+    if (tid == 0) {
+        mbar_init(sm.bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        const uint32_t bytes = static_cast<uint32_t>((2 * (HR + FT) + FT) * kRowWords * 4);
+        mbar_arrive_expect_tx(sm.bar, bytes);
+        if (HR > 0) {
+            tma_load_3d(sm.x1, &th1, sm.bar, cb * FCH, t0 - HR, b);
+            tma_load_3d(sm.x2, &th2, sm.bar, cb * FCH, t0 - HR, b);
+        }
+        tma_load_3d(sm.x1 + HR * kRowWords, &tm1, sm.bar, cb * FCH, t0, b);
+        tma_load_3d(sm.x2 + HR * kRowWords, &tm2, sm.bar, cb * FCH, t0, b);
+        tma_load_3d(sm.x3, &tm3, sm.bar, cb * FCH, t0, b);
+    }
+    // taps -> fp32 [K][lane] while the tiles are in flight
+    for (int idx = tid; idx < K * 32; idx += FW * 32) {
+        const int k = idx >> 5, l = idx & 31;
+        const int c = cb * FCH + 2 * l;
+        float2 t = make_float2(0.f, 0.f);
+        if (c < A.D) {
+            t.x = __uint_as_float(static_cast<uint32_t>(A.taps[static_cast<size_t>(c) * K + k]) << 16);
+            t.y = __uint_as_float(static_cast<uint32_t>(A.taps[static_cast<size_t>(c + 1) * K + k]) << 16);
+        }
+        sm.taps[idx] = t;
+    }
+    const bool ok = mbar_wait_bounded(sm.bar, 0);
+    if (__syncthreads_or(!ok)) {
+        (void)mbar_wait_bounded(sm.bar, 0);
+        return;  // tiles never arrived; output left unwritten
+    }
+
+    // v = x1 * x2 for the halo and the tile; rows before t = 0 from hist_in.
+    const int H = K - 1;
+    for (int r = warp; r < HR + FT; r += FW) {
+        const int t = t0 - HR + r;
+        float2 v;
+        if (t >= 0) {
+            v = __fmul2_rn(bf16x2_to_float2(sm.x1[r * kRowWords + lane]),
+                           bf16x2_to_float2(sm.x2[r * kRowWords + lane]));
+        } else if (t >= -H && A.hist_in != nullptr && ch_ok) {
+            const float *h = A.hist_in + (static_cast<size_t>(b) * H + (H + t)) * A.D + c0;
+            v = *reinterpret_cast<const float2 *>(h);
+        } else {
+            v = make_float2(0.f, 0.f);
+        }
+        sm.v[r * 32 + lane] = v;
+    }
+    __syncthreads();
+
+    float2 acc[FRW];
+#pragma unroll
+    for (int i = 0; i < FRW; ++i) acc[i] = make_float2(0.f, 0.f);
+    const int row0 = HR + warp * FRW;  // v row of this warp's first output
+    int kb = 0;
+    for (; kb + 8 <= K; kb += 8)
+        fir_block<8>(acc, sm.v + (row0 - kb - 7) * 32, sm.taps + kb * 32, lane);
+    switch (K - kb) {
+        case 7: fir_block<7>(acc, sm.v + (row0 - kb - 6) * 32, sm.taps + kb * 32, lane); break;
+        case 6: fir_block<6>(acc, sm.v + (row0 - kb - 5) * 32, sm.taps + kb * 32, lane); break;
+        case 5: fir_block<5>(acc, sm.v + (row0 - kb - 4) * 32, sm.taps + kb * 32, lane); break;
+        case 4: fir_block<4>(acc, sm.v + (row0 - kb - 3) * 32, sm.taps + kb * 32, lane); break;
+        case 3: fir_block<3>(acc, sm.v + (row0 - kb - 2) * 32, sm.taps + kb * 32, lane); break;
+        case 2: fir_block<2>(acc, sm.v + (row0 - kb - 1) * 32, sm.taps + kb * 32, lane); break;
+        case 1: fir_block<1>(acc, sm.v + (row0 - kb) * 32, sm.taps + kb * 32, lane); break;
+        default: break;
+    }
+
+    const float2 dsk = (A.Dskip != nullptr && ch_ok)
+                           ? make_float2(A.Dskip[c0], A.Dskip[c0 + 1])
+                           : make_float2(0.f, 0.f);
+    const int tw0 = t0 + warp * FRW;
+    const int nvalid = min(FRW, A.L - tw0);
+    uint32_t *yrow = reinterpret_cast<uint32_t *>(A.y + (static_cast<size_t>(b) * A.L + tw0) * A.ld_y + c0);
+    const size_t ystride = static_cast<size_t>(A.ld_y) / 2;
+#pragma unroll
+    for (int i = 0; i < FRW; ++i) {
+        if (i < nvalid && ch_ok) {
+            const float2 x3 = bf16x2_to_float2(sm.x3[(warp * FRW + i) * kRowWords + lane]);
+            const float2 v = sm.v[(row0 + i) * 32 + lane];
+            yrow[i * ystride] = float2_to_bf16x2(__ffma2_rn(dsk, v, __fmul2_rn(x3, acc[i])));
+        }
+    }
+}
+
+// hist_out[b][j][c] = v[L-H+j] (from hist_in when that index is negative).
+// One thread per (batch row, channel pair) walks j upward, so reading
+// hist_in[j + L] before writing hist_out[j + L] keeps in-place use safe.
+__global__ void fir_history_kernel(const FirArgs A)
+{
+    const int pairs = A.D / 2;
+    const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= A.B * pairs) return;
+    const int b = idx / pairs;
+    const int c = (idx - b * pairs) * 2;
+    const int H = A.K - 1;
+    for (int j = 0; j < H; ++j) {
+        const int t = A.L - H + j;
+        float2 v;
+        if (t >= 0) {
+            const size_t ix = (static_cast<size_t>(b) * A.L + t) * A.ld_x + c;
+            const uint32_t w1 = *reinterpret_cast<const uint32_t *>(A.x1 + ix);
+            const uint32_t w2 = *reinterpret_cast<const uint32_t *>(A.x2 + ix);
+            v = __fmul2_rn(bf16x2_to_float2(w1), bf16x2_to_float2(w2));
+        } else if (A.hist_in != nullptr) {
+            v = *reinterpret_cast<const float2 *>(A.hist_in + (static_cast<size_t>(b) * H + (H + t)) * A.D + c);
+        } else {
+            v = make_float2(0.f, 0.f);
+        }
+        *reinterpret_cast<float2 *>(A.hist_out + (static_cast<size_t>(b) * H + j) * A.D + c) = v;
+    }
+}
+
+}  // namespace
+
+int launch_fir(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3,
+               const CUtensorMap &h1, const CUtensorMap &h2, const FirArgs &a, cudaStream_t st)
+{
+    int launches = 0;
+    if (a.L > 0) {
+        const size_t smem = fir_smem_bytes(a.HR, a.K);
+        static size_t configured = 0;
+        static int configured_device = -1;
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+        if (configured_device != dev || smem > configured) {
+            const size_t max_smem = fir_smem_bytes(kMaxHalo, HYENA_MAX_TAPS);
+            if (cudaFuncSetAttribute(fir_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(max_smem)) != cudaSuccess)
+                return -1;
+            configured = max_smem;
+            configured_device = dev;
+        }
+        const dim3 grid((a.D + FCH - 1) / FCH, (a.L + FT - 1) / FT, a.B);
+        fir_kernel<<<grid, FW * 32, smem, st>>>(m1, m2, m3, h1, h2, a);
+        if (cudaGetLastError() != cudaSuccess) return -1;
+        ++launches;
+    }
+    if (a.hist_out != nullptr && a.K > 1) {
+        const int threads = a.B * (a.D / 2);
+        fir_history_kernel<<<(threads + 255) / 256, 256, 0, st>>>(a);
+        if (cudaGetLastError() != cudaSuccess) return -1;
+        ++launches;
+    }
+    return launches;
+}
+
+}  // namespace hyena

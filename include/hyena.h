@@ -1,0 +1,165 @@
+/*
+ * hyena.h -- C ABI of libhyena_b200.so: the gated Hyena cascade operator of
+ * StripedHyena 2 / Evo 2 on NVIDIA B200 (sm_100a).
+ *
+ *   v[t]    = x1[t] * x2[t]
+ *   conv[t] = (h_c * v)[t]               causal, depthwise (one filter per channel)
+ *   y[t]    = x3[t] * conv[t] + Dskip[c] * v[t]
+ *
+ * x1, x2, x3 are the three slices of the Hyena input projection and y is the
+ * gated filter output that feeds out_proj (evo2_flash README, hook table rows
+ * "blocks.N.projections" and "blocks.N.filter").  The filter h_c is either
+ * explicit and short (hcs: 7 taps, hcm: 128 taps) or the long modal-form hcl
+ * filter h_c[t] = sum_n R[c,n] exp(a[c,n] t) with fp32 log-poles a and
+ * residues R (Evo2-7B-262K model card, §Architecture and §Implementation
+ * Notes).  Long sequences can be fed in chunks: the modal state (hcl) or the
+ * FIR window (hcs/hcm) is carried from one call to the next, and every
+ * position of every chunk is produced (Evo2-7B-262K model card, "Custom
+ * cache"; turboquant-evo2-int4 model card, §"Important: a correctness fix
+ * comes with this" and §"Chunk size").
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are bf16 (passed as hyena_bf16_t bit patterns), layout
+ *     [B, L, D], channel-contiguous: element (b, t, c) sits at
+ *     (b * L + t) * ld + c.  ld >= D is a row stride in elements, so x1, x2,
+ *     x3 may be three views of one [B, L, 3D] projection output (ld = 3D).
+ *   - Every device pointer is a device address owned by the caller; the
+ *     library allocates no device memory.  Pointers must be 16-byte aligned,
+ *     D and ld must be multiples of 8.
+ *   - Arithmetic is fp32 (v is exact in fp32); y is rounded once to bf16
+ *     (round to nearest even).  NaN and Inf propagate.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Argument checks run on the host before any launch;
+ *     on failure nothing is launched and a non-zero status is returned.
+ *     No C++ exception crosses this interface.
+ *   - y must not overlap x1, x2, x3.  state_in may equal state_out and
+ *     hist_in may equal hist_out (in-place chunking).
+ */
+#ifndef HYENA_B200_H
+#define HYENA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t hyena_bf16_t; /* bf16 bit pattern */
+
+typedef enum {
+    HYENA_OK = 0,
+    HYENA_ERR_INVALID_ARG = 1, /* null pointer, bad size or shape            */
+    HYENA_ERR_ALIGNMENT = 2,   /* pointer / D / ld not aligned as required   */
+    HYENA_ERR_UNSUPPORTED = 3, /* N or K outside the supported range         */
+    HYENA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed       */
+    HYENA_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out         */
+    HYENA_ERR_WORKSPACE = 6    /* workspace missing or too small             */
+} hyena_status_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *hyena_status_string(hyena_status_t s);
+
+/* Version of this interface (major * 100 + minor). */
+int hyena_abi_version(void);
+
+/* Largest supported number of modes N and of FIR taps K. */
+#define HYENA_MAX_MODES 16
+#define HYENA_MAX_TAPS 128
+
+/*
+ * Explicit short causal FIR (hcs, K = 7; hcm, K = 128): Evo2-7B-262K model
+ * card, §Implementation Notes ("Block dispatch": FIR cascades with inner
+ * lengths 7 and 128; "Custom cache": the FIR window carried between steps).
+ *
+ *   conv[t] = sum_{k<K} taps[c*K + k] * v[t-k]     (lag order)
+ *
+ * taps      [D, K] bf16, device.  1 <= K <= HYENA_MAX_TAPS.
+ * Dskip     [D] fp32, device, or NULL (no skip term).
+ * hist_in   [B, K-1, D] fp32, device, or NULL: the K-1 values of v that
+ *           precede t = 0, oldest first (hist_in[b][K-1-j][c] = v[-j]).
+ *           NULL means zeros.
+ * hist_out  [B, K-1, D] fp32, device, or NULL: receives the last K-1
+ *           values of v of the sequence continued by this call, in the same
+ *           layout, ready to be passed as the next call's hist_in.
+ * L == 0 is valid: y is untouched and hist_out receives hist_in (or zeros).
+ */
+hyena_status_t hyena_short_conv(const hyena_bf16_t *x1, const hyena_bf16_t *x2,
+                                const hyena_bf16_t *x3, int64_t ld_x,
+                                const hyena_bf16_t *taps, const float *Dskip,
+                                hyena_bf16_t *y, int64_t ld_y,
+                                const float *hist_in, float *hist_out,
+                                int B, int L, int D, int K, void *stream);
+
+/*
+ * Bytes of device workspace hyena_modal_long_conv needs for B, D, N
+ * (independent of L).  Returns 0 for invalid sizes.
+ */
+size_t hyena_modal_long_conv_workspace_size(int B, int D, int N);
+
+/*
+ * Zero-fills a workspace (asynchronously on `stream`).  A workspace must be
+ * zero-filled once before its first use; afterwards it can be reused by any
+ * number of calls whose workspace size fits, on one stream at a time.
+ */
+hyena_status_t hyena_modal_workspace_init(void *workspace, size_t workspace_bytes,
+                                          void *stream);
+
+/*
+ * Long modal-form filter (hcl): Evo2-7B-262K model card, §Architecture
+ * (log_poles / residues kept in fp32) and §Implementation Notes (hcl as a
+ * modal-form IIR; "Custom cache" for the carried IIR state).
+ *
+ *   h_c[t] = sum_{n<N} residues[c*N+n] * exp(log_poles[c*N+n] * t),  t >= 0
+ *
+ * log_poles, residues  [D, N] fp32, device.  1 <= N <= HYENA_MAX_MODES.
+ *           Any real log-pole is accepted; the pages' filters have a < 0.
+ * Dskip     [D] fp32, device, or NULL (no skip term).
+ * state_in  [B, D, N] fp32, device, or NULL (zeros): the per-mode state
+ *           s_n = sum_{s<=t} exp(a_n (t-s)) v[s] after the last token of
+ *           the previous chunk.  It contributes
+ *           sum_n R_n exp(a_n (t+1)) state_in[n] to conv[t].
+ * state_out [B, D, N] fp32, device, or NULL: the state after token L-1.
+ * workspace device memory of at least
+ *           hyena_modal_long_conv_workspace_size(B, D, N) bytes, zero-filled
+ *           once by hyena_modal_workspace_init.  Calls sharing a workspace
+ *           must not overlap in time (same stream or synchronised).
+ * L == 0 is valid: y is untouched and state_out receives state_in (or zeros).
+ * Device-side waits are bounded; if one runs out the call's output is
+ * invalid and hyena_workspace_check reports HYENA_ERR_TIMEOUT.
+ */
+hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t *x2,
+                                     const hyena_bf16_t *x3, int64_t ld_x,
+                                     const float *log_poles, const float *residues,
+                                     const float *Dskip,
+                                     hyena_bf16_t *y, int64_t ld_y,
+                                     const float *state_in, float *state_out,
+                                     int B, int L, int D, int N,
+                                     void *workspace, size_t workspace_bytes,
+                                     void *stream);
+
+/*
+ * Zero-fills a modal state [B, D, N] fp32 (the state before the first token
+ * of a sequence): the start of chunked prefill.
+ */
+hyena_status_t hyena_modal_state_init(float *state, int B, int D, int N, void *stream);
+
+/*
+ * Synchronises `stream`, then reports (and clears) a device-side error that
+ * calls using this workspace recorded: HYENA_ERR_TIMEOUT if a bounded wait
+ * ran out, HYENA_OK otherwise.
+ */
+hyena_status_t hyena_workspace_check(void *workspace, void *stream);
+
+/*
+ * Number of kernels (and memset/copy nodes) the most recent successful call
+ * of each entry point on this thread enqueued; used by benchmarks to report
+ * launch counts.
+ */
+int hyena_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HYENA_B200_H */

@@ -1,0 +1,116 @@
+"""The C-ABI library loads on a host without a GPU, exports every entry point
+that include/hyena.h declares, and rejects bad arguments on the host before
+touching the device (no compute call is made here).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import hyena_long_convolution_b200 as hy
+from hyena_long_convolution_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hyena.h")
+
+OK, INVALID, ALIGN, UNSUP, CUDA, TIMEOUT, WORKSPACE = range(7)
+A = 0x10000  # a 16-byte-aligned fake device address; never dereferenced here
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hyena_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_and_binding_agree():
+    names = declared_functions()
+    assert names, "no declarations parsed"
+    assert sorted(_lib.SIGNATURES) == names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = hy.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings_and_version():
+    lib = hy.lib()
+    for code, name in _lib.STATUS.items():
+        assert lib.hyena_status_string(code).decode() == name
+    assert lib.hyena_status_string(99).decode() == "HYENA_ERR_UNKNOWN"
+    assert lib.hyena_abi_version() == 100
+
+
+def test_workspace_size():
+    lib = hy.lib()
+    assert lib.hyena_modal_long_conv_workspace_size(0, 64, 8) == 0
+    assert lib.hyena_modal_long_conv_workspace_size(1, 64, 0) == 0
+    assert lib.hyena_modal_long_conv_workspace_size(1, 64, hy.MAX_MODES + 1) == 0
+    a = lib.hyena_modal_long_conv_workspace_size(1, 4096, 16)
+    b = lib.hyena_modal_long_conv_workspace_size(2, 4096, 16)
+    c = lib.hyena_modal_long_conv_workspace_size(1, 4096, 8)
+    assert 0 < c < a < b
+    assert a % 256 == 0
+    # independent of the sequence length by construction: no L argument
+    assert a < 64 << 20
+
+
+def modal(lib, **kw):
+    args = dict(x1=A, x2=A, x3=A, ld_x=64, lp=A, res=A, ds=None, y=A + 4096, ld_y=64,
+                s_in=None, s_out=None, B=1, L=16, D=64, N=8, ws=None, ws_bytes=0, st=None)
+    args.update(kw)
+    return lib.hyena_modal_long_conv(args["x1"], args["x2"], args["x3"], args["ld_x"], args["lp"],
+                                     args["res"], args["ds"], args["y"], args["ld_y"], args["s_in"],
+                                     args["s_out"], args["B"], args["L"], args["D"], args["N"],
+                                     args["ws"], args["ws_bytes"], args["st"])
+
+
+def fir(lib, **kw):
+    args = dict(x1=A, x2=A, x3=A, ld_x=64, taps=A, ds=None, y=A + 4096, ld_y=64, h_in=None,
+                h_out=None, B=1, L=16, D=64, K=7, st=None)
+    args.update(kw)
+    return lib.hyena_short_conv(args["x1"], args["x2"], args["x3"], args["ld_x"], args["taps"],
+                                args["ds"], args["y"], args["ld_y"], args["h_in"], args["h_out"],
+                                args["B"], args["L"], args["D"], args["K"], args["st"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), INVALID), (dict(L=-1), INVALID), (dict(D=0), INVALID),
+    (dict(x1=None), INVALID), (dict(y=None), INVALID), (dict(lp=None), INVALID),
+    (dict(res=None), INVALID), (dict(N=0), INVALID), (dict(N=17), UNSUP),
+    (dict(ld_x=32), INVALID), (dict(ld_y=60), INVALID), (dict(D=60, ld_x=64, ld_y=64), ALIGN),
+    (dict(ld_x=68), ALIGN), (dict(x2=A + 2), ALIGN), (dict(y=A + 8), ALIGN),
+    (dict(s_in=A + 4), ALIGN), (dict(ds=A + 4), ALIGN),
+    (dict(ws=None), WORKSPACE), (dict(ws=A, ws_bytes=1024), WORKSPACE),
+])
+def test_modal_rejects_bad_arguments(kw, code):
+    assert modal(hy.lib(), **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), INVALID), (dict(L=-5), INVALID), (dict(x3=None), INVALID), (dict(taps=None), INVALID),
+    (dict(K=0), INVALID), (dict(K=129), UNSUP), (dict(ld_x=8), INVALID), (dict(x1=A + 6), ALIGN),
+    (dict(taps=A + 2), ALIGN), (dict(h_in=A + 4), ALIGN), (dict(D=12, ld_x=16, ld_y=16), ALIGN),
+])
+def test_short_conv_rejects_bad_arguments(kw, code):
+    assert fir(hy.lib(), **kw) == code
+
+
+def test_other_entry_points_reject_bad_arguments():
+    lib = hy.lib()
+    assert lib.hyena_modal_state_init(None, 1, 64, 8, None) == INVALID
+    assert lib.hyena_modal_state_init(A, 0, 64, 8, None) == INVALID
+    assert lib.hyena_modal_workspace_init(None, 100, None) == INVALID
+    assert lib.hyena_modal_workspace_init(A, 0, None) == INVALID
+    assert lib.hyena_workspace_check(None, None) == INVALID
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "SO", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(ImportError):
+        _lib.lib()

@@ -31,6 +31,7 @@ SIGNATURES = {
     "hyena_status_string": (ctypes.c_char_p, [_I]),
     "hyena_abi_version": (_I, []),
     "hyena_last_launch_count": (_I, []),
+    "hyena_last_error_message": (ctypes.c_char_p, []),
     "hyena_short_conv": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I64, _P, _P, _I, _I, _I, _I, _P]),
     "hyena_modal_long_conv_workspace_size": (_SZ, [_I, _I, _I]),
     "hyena_modal_workspace_init": (_I, [_P, _SZ, _P]),
@@ -68,4 +69,7 @@ def lib() -> ctypes.CDLL:
 
 def check(fn: str, status: int) -> None:
     if status != 0:
-        raise HyenaError(fn, status)
+        err = HyenaError(fn, status)
+        if status == 4:  # HYENA_ERR_CUDA: attach the failing runtime call
+            err.args = (f"{err.args[0]} ({lib().hyena_last_error_message().decode()})",)
+        raise err

@@ -3,7 +3,7 @@
 // kernels.  Nothing here computes any part of the operator.
 #include <cudaTypedefs.h>
 
-#include <atomic>
+#include <cstdio>
 #include <mutex>
 
 #include "hyena_internal.h"
@@ -13,6 +13,7 @@ namespace hyena {
 namespace {
 
 thread_local int g_last_launches = 0;
+thread_local char g_last_error[256] = "no error";
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -43,6 +44,21 @@ bool encode_bf16_map(CUtensorMap *m, const void *base, int B, int L, int D, long
                                 strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                                 CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// 2-D fp32 tensor map over a row-major [rows, cols] table, box [rows x 64].
+bool encode_f32_table_map(CUtensorMap *m, const void *base, int rows, int cols)
+{
+    std::call_once(g_encode_once, resolve_encode);
+    if (g_encode == nullptr) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 4};
+    cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(rows)};
+    cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides,
+                                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -78,24 +94,25 @@ hyena_status_t copy_or_zero(float *dst, const float *src, size_t bytes, cudaStre
 
 }  // namespace
 
+void record_cuda_error(cudaError_t e, const char *where)
+{
+    snprintf(g_last_error, sizeof g_last_error, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
 ModalLayout modal_layout(int B, int D, int N)
 {
     ModalLayout L;
     L.NP = modal_padded_modes(N);
     L.nCB = (D + MCH - 1) / MCH;
     L.Dp = L.nCB * MCH;
-    const size_t tab = static_cast<size_t>(L.NP) * L.Dp * sizeof(float);
+    const size_t row = static_cast<size_t>(L.Dp) * sizeof(float);
     size_t off = 0;
     L.off_hdr = off;
     off += 256;
-    L.off_cP = off;
-    off = align256(off + tab);
-    L.off_cR = off;
-    off = align256(off + tab);
-    L.off_cPw = off;
-    off = align256(off + tab * (MW + 1));
-    L.off_cDs = off;
-    off = align256(off + static_cast<size_t>(L.Dp) * sizeof(float));
+    L.off_coef = off;
+    off = align256(off + row * modal_coef_rows(L.NP));
+    L.off_pT = off;
+    off = align256(off + row * L.NP);
     const size_t chains = static_cast<size_t>(B) * L.nCB;
     L.off_flags = off;
     off = align256(off + chains * MRING * sizeof(unsigned long long));
@@ -128,6 +145,8 @@ const char *hyena_status_string(hyena_status_t s)
 int hyena_abi_version(void) { return 100; }
 
 int hyena_last_launch_count(void) { return g_last_launches; }
+
+const char *hyena_last_error_message(void) { return g_last_error; }
 
 hyena_status_t hyena_short_conv(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
                                 int64_t ld_x, const hyena_bf16_t *taps, const float *Dskip,
@@ -230,6 +249,8 @@ hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t 
 
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     ModalArgs a{};
+    a.x3 = x3;
+    a.ld_x = ld_x;
     a.y = y;
     a.ld_y = ld_y;
     a.state_in = state_in;
@@ -241,10 +262,7 @@ hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t 
     a.nCB = lay.nCB;
     a.Dp = lay.Dp;
     a.nUnits = static_cast<unsigned int>(units);
-    a.cP = reinterpret_cast<const float *>(ws + lay.off_cP);
-    a.cR = reinterpret_cast<const float *>(ws + lay.off_cR);
-    a.cPw = reinterpret_cast<const float *>(ws + lay.off_cPw);
-    a.cDs = reinterpret_cast<const float *>(ws + lay.off_cDs);
+    a.cPT = reinterpret_cast<const float *>(ws + lay.off_pT);
     a.flags = reinterpret_cast<unsigned long long *>(ws + lay.off_flags);
     a.slots = reinterpret_cast<float *>(ws + lay.off_slots);
     a.hdr = reinterpret_cast<unsigned int *>(ws + lay.off_hdr);
@@ -256,16 +274,14 @@ hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t 
     sy.D = D;
     sy.N = N;
     sy.Dp = lay.Dp;
-    sy.cP = reinterpret_cast<float *>(ws + lay.off_cP);
-    sy.cR = reinterpret_cast<float *>(ws + lay.off_cR);
-    sy.cPw = reinterpret_cast<float *>(ws + lay.off_cPw);
-    sy.cDs = reinterpret_cast<float *>(ws + lay.off_cDs);
+    sy.coef = reinterpret_cast<float *>(ws + lay.off_coef);
+    sy.cPT = reinterpret_cast<float *>(ws + lay.off_pT);
 
-    CUtensorMap m1, m2, m3;
+    CUtensorMap m1, m2, mc;
     if (!encode_bf16_map(&m1, x1, B, L, D, ld_x, MT) || !encode_bf16_map(&m2, x2, B, L, D, ld_x, MT) ||
-        !encode_bf16_map(&m3, x3, B, L, D, ld_x, MT))
+        !encode_f32_table_map(&mc, ws + lay.off_coef, modal_coef_rows(lay.NP), lay.Dp))
         return HYENA_ERR_CUDA;
-    const int n = launch_modal(m1, m2, m3, a, sy, lay.NP, s);
+    const int n = launch_modal(m1, m2, mc, a, sy, lay.NP, s);
     if (n < 0) return HYENA_ERR_CUDA;
     g_last_launches = n;
     return HYENA_OK;

@@ -11,6 +11,19 @@
 
 namespace hyena {
 
+// Remembers the most recent failing CUDA call of this thread (reported by
+// hyena_last_error_message).
+void record_cuda_error(cudaError_t e, const char *where);
+
+#define HYENA_TRY(call, where)                       \
+    do {                                             \
+        const cudaError_t e_ = (call);               \
+        if (e_ != cudaSuccess) {                     \
+            ::hyena::record_cuda_error(e_, where);   \
+            return -1;                               \
+        }                                            \
+    } while (0)
+
 // ---------------------------------------------------------------- modal scan
 // Work unit: MCH channels x MT tokens of one batch row.  One CTA of MW warps
 // processes a unit; warp w owns tokens [w*MS, (w+1)*MS) of it and lane l the
@@ -24,15 +37,20 @@ constexpr int MLB = 16;    // deepest look-back, in units
 
 inline int modal_padded_modes(int N) { return N <= 4 ? 4 : (N <= 8 ? 8 : 16); }
 
+// Coefficient block per channel block, staged with each unit's tiles:
+// rows [0, NP) p = exp(a), [NP, 2NP) residues R, [2NP, 3NP) p^MS, row 3NP Dskip.
+inline int modal_coef_rows(int NP) { return 3 * NP + 1; }
+
 struct ModalLayout {
     int NP = 0, nCB = 0, Dp = 0;
-    size_t off_hdr = 0, off_cP = 0, off_cR = 0, off_cPw = 0, off_cDs = 0, off_flags = 0,
-           off_slots = 0, total = 0;
+    size_t off_hdr = 0, off_coef = 0, off_pT = 0, off_flags = 0, off_slots = 0, total = 0;
 };
 
 ModalLayout modal_layout(int B, int D, int N);
 
 struct ModalArgs {
+    const uint16_t *x3;
+    long long ld_x;
     uint16_t *y;
     long long ld_y;
     const float *state_in;
@@ -40,24 +58,23 @@ struct ModalArgs {
     int B, L, D, N;
     int nCB, Dp;
     unsigned int nUnits;
-    const float *cP;    // [NP][Dp]  exp(a)
-    const float *cR;    // [NP][Dp]  residues
-    const float *cPw;   // [MW+1][NP][Dp]  exp(a * MS * w)
-    const float *cDs;   // [Dp]  skip
+    const float *cPT;           // [NP][Dp]  p^MT
     unsigned long long *flags;  // [B*nCB][MRING]
-    float *slots;       // [B*nCB][MRING][2][NP][MCH]
-    unsigned int *hdr;  // [0] ticket, [1] finished CTAs, [2] error bits, [3] epoch
+    float *slots;               // [B*nCB][MRING][2][NP][MCH]
+    unsigned int *hdr;          // [0] ticket, [1] finished CTAs, [2] error bits, [3] epoch
 };
 
 struct ModalSynthArgs {
     const float *log_poles, *residues, *Dskip;
     int D, N, Dp;
-    float *cP, *cR, *cPw, *cDs;
+    float *coef;  // [3NP+1][Dp]
+    float *cPT;   // [NP][Dp]
 };
 
 // Launches the coefficient-synthesis kernel and the scan kernel; returns the
-// number of launches enqueued or a negative value on a CUDA error.
-int launch_modal(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3,
+// number of launches enqueued or a negative value on a CUDA error.  mc is the
+// tensor map of the coefficient table (fp32 [3NP+1][Dp], box [3NP+1 x 64]).
+int launch_modal(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &mc,
                  const ModalArgs &a, const ModalSynthArgs &s, int NP, cudaStream_t st);
 
 // ---------------------------------------------------------------- short FIR

@@ -212,24 +212,24 @@ int launch_fir(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &
         static size_t configured = 0;
         static int configured_device = -1;
         int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+        HYENA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
         if (configured_device != dev || smem > configured) {
             const size_t max_smem = fir_smem_bytes(kMaxHalo, HYENA_MAX_TAPS);
-            if (cudaFuncSetAttribute(fir_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(max_smem)) != cudaSuccess)
-                return -1;
+            HYENA_TRY(cudaFuncSetAttribute(fir_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(max_smem)),
+                      "fir: set max dynamic shared memory");
             configured = max_smem;
             configured_device = dev;
         }
         const dim3 grid((a.D + FCH - 1) / FCH, (a.L + FT - 1) / FT, a.B);
         fir_kernel<<<grid, FW * 32, smem, st>>>(m1, m2, m3, h1, h2, a);
-        if (cudaGetLastError() != cudaSuccess) return -1;
+        HYENA_TRY(cudaGetLastError(), "fir launch");
         ++launches;
     }
     if (a.hist_out != nullptr && a.K > 1) {
         const int threads = a.B * (a.D / 2);
         fir_history_kernel<<<(threads + 255) / 256, 256, 0, st>>>(a);
-        if (cudaGetLastError() != cudaSuccess) return -1;
+        HYENA_TRY(cudaGetLastError(), "fir history launch");
         ++launches;
     }
     return launches;

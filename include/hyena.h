@@ -158,6 +158,13 @@ hyena_status_t hyena_workspace_check(void *workspace, void *stream);
  */
 int hyena_last_launch_count(void);
 
+/*
+ * Text describing the most recent failing CUDA runtime call made by an entry
+ * point on this thread (the cause behind HYENA_ERR_CUDA); a static,
+ * thread-local string, never NULL.
+ */
+const char *hyena_last_error_message(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -47,21 +47,6 @@ bool encode_bf16_map(CUtensorMap *m, const void *base, int B, int L, int D, long
     return r == CUDA_SUCCESS;
 }
 
-// 2-D fp32 tensor map over a row-major [rows, cols] table, box [rows x 64].
-bool encode_f32_table_map(CUtensorMap *m, const void *base, int rows, int cols)
-{
-    std::call_once(g_encode_once, resolve_encode);
-    if (g_encode == nullptr) return false;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 4};
-    cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(rows)};
-    cuuint32_t estr[2] = {1u, 1u};
-    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides,
-                                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 hyena_status_t check_x(const void *x1, const void *x2, const void *x3, long long ld_x, const void *y,
@@ -111,13 +96,11 @@ ModalLayout modal_layout(int B, int D, int N)
     off += 256;
     L.off_coef = off;
     off = align256(off + row * modal_coef_rows(L.NP));
-    L.off_pT = off;
-    off = align256(off + row * L.NP);
     const size_t chains = static_cast<size_t>(B) * L.nCB;
     L.off_flags = off;
     off = align256(off + chains * MRING * sizeof(unsigned long long));
     L.off_slots = off;
-    off = align256(off + chains * MRING * 2 * L.NP * MCH * sizeof(float));
+    off = align256(off + chains * MRING * (MGMAX + 1) * L.NP * MCH * sizeof(float));
     L.total = off;
     return L;
 }
@@ -244,8 +227,7 @@ hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t 
     if (workspace == nullptr || workspace_bytes < lay.total) return HYENA_ERR_WORKSPACE;
     if (!aligned16(workspace)) return HYENA_ERR_ALIGNMENT;
     const long long nseg = (static_cast<long long>(L) + MT - 1) / MT;
-    const long long units = nseg * B * lay.nCB;
-    if (units >= (1ll << 31)) return HYENA_ERR_UNSUPPORTED;
+    if (nseg * B * lay.nCB >= (1ll << 31)) return HYENA_ERR_UNSUPPORTED;
 
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     ModalArgs a{};
@@ -261,8 +243,8 @@ hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t 
     a.N = N;
     a.nCB = lay.nCB;
     a.Dp = lay.Dp;
-    a.nUnits = static_cast<unsigned int>(units);
-    a.cPT = reinterpret_cast<const float *>(ws + lay.off_pT);
+    a.units = static_cast<int>(nseg);
+    a.coef = reinterpret_cast<const float *>(ws + lay.off_coef);
     a.flags = reinterpret_cast<unsigned long long *>(ws + lay.off_flags);
     a.slots = reinterpret_cast<float *>(ws + lay.off_slots);
     a.hdr = reinterpret_cast<unsigned int *>(ws + lay.off_hdr);
@@ -275,13 +257,12 @@ hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t 
     sy.N = N;
     sy.Dp = lay.Dp;
     sy.coef = reinterpret_cast<float *>(ws + lay.off_coef);
-    sy.cPT = reinterpret_cast<float *>(ws + lay.off_pT);
 
-    CUtensorMap m1, m2, mc;
-    if (!encode_bf16_map(&m1, x1, B, L, D, ld_x, MT) || !encode_bf16_map(&m2, x2, B, L, D, ld_x, MT) ||
-        !encode_f32_table_map(&mc, ws + lay.off_coef, modal_coef_rows(lay.NP), lay.Dp))
+    CUtensorMap m1, m2, m3;
+    if (!encode_bf16_map(&m1, x1, B, L, D, ld_x, MCK) || !encode_bf16_map(&m2, x2, B, L, D, ld_x, MCK) ||
+        !encode_bf16_map(&m3, x3, B, L, D, ld_x, MCK))
         return HYENA_ERR_CUDA;
-    const int n = launch_modal(m1, m2, mc, a, sy, lay.NP, s);
+    const int n = launch_modal(m1, m2, m3, a, sy, lay.NP, s);
     if (n < 0) return HYENA_ERR_CUDA;
     g_last_launches = n;
     return HYENA_OK;

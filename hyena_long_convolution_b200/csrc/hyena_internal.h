@@ -25,25 +25,27 @@ void record_cuda_error(cudaError_t e, const char *where);
     } while (0)
 
 // ---------------------------------------------------------------- modal scan
-// Work unit: MCH channels x MT tokens of one batch row.  One CTA of MW warps
-// processes a unit; warp w owns tokens [w*MS, (w+1)*MS) of it and lane l the
-// channel pair (2l, 2l+1).
+// A chain is the sequence of MCH channels of one batch row over time.  A unit
+// is MT consecutive tokens of a chain, swept by one warp (lane l owns the
+// channel pair 2l, 2l+1); a group is G consecutive units handled by one CTA of
+// G compute warps plus a control warp.  Tiles stream through shared memory in
+// chunks of MCK rows.
 constexpr int MCH = 64;
 constexpr int MT = 128;
-constexpr int MW = 8;
-constexpr int MS = MT / MW;
-constexpr int MRING = 32;  // ring slots per (batch row, channel block) chain
-constexpr int MLB = 16;    // deepest look-back, in units
+constexpr int MCK = 16;
+constexpr int MRING = 16;  // group slots per chain
+constexpr int MLB = 8;     // deepest look-back, in groups
+constexpr int MGMAX = 4;   // largest group (slots are sized for it)
 
 inline int modal_padded_modes(int N) { return N <= 4 ? 4 : (N <= 8 ? 8 : 16); }
 
-// Coefficient block per channel block, staged with each unit's tiles:
-// rows [0, NP) p = exp(a), [NP, 2NP) residues R, [2NP, 3NP) p^MS, row 3NP Dskip.
+// Coefficient table [3NP+1][Dp]: rows [0, NP) p = exp(a), [NP, 2NP) residues,
+// row 2NP Dskip, rows [2NP+1, 3NP+1) p^MT.
 inline int modal_coef_rows(int NP) { return 3 * NP + 1; }
 
 struct ModalLayout {
     int NP = 0, nCB = 0, Dp = 0;
-    size_t off_hdr = 0, off_coef = 0, off_pT = 0, off_flags = 0, off_slots = 0, total = 0;
+    size_t off_hdr = 0, off_coef = 0, off_flags = 0, off_slots = 0, total = 0;
 };
 
 ModalLayout modal_layout(int B, int D, int N);
@@ -57,25 +59,25 @@ struct ModalArgs {
     float *state_out;
     int B, L, D, N;
     int nCB, Dp;
-    unsigned int nUnits;
-    const float *cPT;           // [NP][Dp]  p^MT
+    int units;                  // units per chain, ceil(L / MT)
+    unsigned int nGroups;       // groups over all chains
+    const float *coef;          // [3NP+1][Dp]
     unsigned long long *flags;  // [B*nCB][MRING]
-    float *slots;               // [B*nCB][MRING][2][NP][MCH]
+    float *slots;               // [B*nCB][MRING][MGMAX+1][NP][MCH]
     unsigned int *hdr;          // [0] ticket, [1] finished CTAs, [2] error bits, [3] epoch
 };
 
 struct ModalSynthArgs {
     const float *log_poles, *residues, *Dskip;
     int D, N, Dp;
-    float *coef;  // [3NP+1][Dp]
-    float *cPT;   // [NP][Dp]
+    float *coef;
 };
 
 // Launches the coefficient-synthesis kernel and the scan kernel; returns the
-// number of launches enqueued or a negative value on a CUDA error.  mc is the
-// tensor map of the coefficient table (fp32 [3NP+1][Dp], box [3NP+1 x 64]).
-int launch_modal(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &mc,
-                 const ModalArgs &a, const ModalSynthArgs &s, int NP, cudaStream_t st);
+// number of launches enqueued or a negative value on a CUDA error.  The three
+// tensor maps cover x1, x2, x3 with [MCK x MCH] boxes.
+int launch_modal(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3,
+                 ModalArgs a, const ModalSynthArgs &s, int NP, cudaStream_t st);
 
 // ---------------------------------------------------------------- short FIR
 constexpr int FCH = 64;   // channels per CTA

@@ -33,9 +33,11 @@
 //            from L2) and reruns the recurrences from C_j, emitting
 //            y = x3 * sum_n R_n s_n + Dskip v as coalesced 128-byte rows
 //            (2N FMAs per token).
-// Each compute warp streams its rows through its own ring of TMA-filled
-// chunk buffers, issued several chunks ahead; several CTAs share an SM, so one
-// CTA's look-back overlaps the others' sweeps.
+// Each compute warp streams its rows through its own ring of chunk buffers,
+// filled several chunks ahead by the CTA's producer warp with TMA; the compute
+// warps publish their own aggregates (the control warp only raises the flag),
+// and several CTAs share an SM, so one CTA's look-back overlaps the others'
+// sweeps.
 //
 // Ring of slots: each chain owns MRING group slots; group s writes slot
 // s % MRING.  The look-back never goes deeper than MLB groups (it waits for an
@@ -62,16 +64,18 @@ constexpr int kChunksPerGroup = 2 * kChunksPerSweep;
 template <int G>
 struct GroupTraits {
     static constexpr int kRing = G >= 4 ? 4 : 3;  // chunk buffers per compute warp
-    static constexpr int kThreads = 32 * (G + 1);
-    static constexpr int kCtasPerSm = 8 / G;
+    static constexpr int kThreads = 32 * (G + 2);  // compute warps, control warp, producer warp
+    static constexpr int kCtasPerSm = G >= 4 ? 2 : 3;
 };
 
 template <int NP, int G>
 struct GroupSmem {
     uint32_t ring[G][GroupTraits<G>::kRing][3][kChunkWords];  // x1, x2, x3 chunks per compute warp
     float2 ac[G][NP * 32];       // unit aggregate A_j, then (in place) the carry C_j
-    uint64_t full[G][GroupTraits<G>::kRing];
-    uint64_t gready[2];          // group id known (control -> compute)
+    uint64_t full[G][GroupTraits<G>::kRing];   // chunk landed (producer TMA -> compute)
+    uint64_t empty[G][GroupTraits<G>::kRing];  // chunk consumed (compute -> producer)
+    uint64_t gready[2];          // group id known (control -> compute, producer)
+    uint64_t slotok[2];          // ring slot may be written (control -> compute)
     uint64_t adone[2];           // aggregates written (compute -> control)
     uint64_t cdone[2];           // carries written (control -> compute)
     int gid[2];
@@ -213,7 +217,7 @@ __device__ void control_warp(GroupSmem<NP, G> &sm, const ModalArgs &A, unsigned 
         load_rows<NP>(pT, A.coef, 2 * NP + 1, A.Dp, c0);
 
         // Ring guard: groups s-MRING .. s-MLB must be finished before this
-        // group writes slot s % MRING.
+        // group's slot s % MRING is written.
         if (s >= static_cast<unsigned int>(MRING) && lane <= MRING - MLB) {
             const unsigned int jg = s - MRING + lane;
             const unsigned long long need = flag_word(epoch, jg, true) & 0xffffffffull;
@@ -222,19 +226,15 @@ __device__ void control_warp(GroupSmem<NP, G> &sm, const ModalArgs &A, unsigned 
             });
         }
         __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.slotok[k & 1]);
 
         // ---------------- publish the group's unit aggregates (flag AGG)
+        // Each compute warp wrote its unit's aggregate to the slot and fenced
+        // before arriving; the release store orders all of them before the
+        // flag for any reader that acquires it.
         (void)mbar_wait_or_flag(&sm.adone[k & 1], (k >> 1) & 1, A.hdr);
-        if (s > 0u && has_successor) {
-            for (int w = 0; w < G; ++w) {
-#pragma unroll
-                for (int n = 0; n < NP; ++n)
-                    *reinterpret_cast<float2 *>(slot + (static_cast<size_t>(w) * NP + n) * MCH) = sm.ac[w][n * 32 + lane];
-            }
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) st_release_u64(chain_flags + (s % MRING), flag_word(epoch, s, false));
-        }
+        if (s > 0u && has_successor && lane == 0)
+            st_release_u64(chain_flags + (s % MRING), flag_word(epoch, s, false));
 
         // ---------------- look-back: the carry into the group's first unit
         float2 C[NP];
@@ -298,13 +298,18 @@ __device__ void control_warp(GroupSmem<NP, G> &sm, const ModalArgs &A, unsigned 
             // (the canonical chain).
             for (unsigned int jg = jincl + 1u; ok && jg < s; ++jg) {
                 const float *src = chain_slots + static_cast<size_t>(jg % MRING) * slot_floats + 2 * lane;
-                for (int w = 0; w < G; ++w) {
-                    float2 a[NP];
+                for (int w = 0; w < G; w += 2) {
+                    // two units' aggregates in flight at once
+                    float2 a[NP], b2[NP];
 #pragma unroll
-                    for (int n = 0; n < NP; ++n)
+                    for (int n = 0; n < NP; ++n) {
                         a[n] = __ldcg(reinterpret_cast<const float2 *>(src + (static_cast<size_t>(w) * NP + n) * MCH));
+                        b2[n] = __ldcg(reinterpret_cast<const float2 *>(src + (static_cast<size_t>(w + 1) * NP + n) * MCH));
+                    }
 #pragma unroll
                     for (int n = 0; n < NP; ++n) C[n] = __ffma2_rn(pT[n], C[n], a[n]);
+#pragma unroll
+                    for (int n = 0; n < NP; ++n) C[n] = __ffma2_rn(pT[n], C[n], b2[n]);
                 }
             }
         }
@@ -349,60 +354,51 @@ __device__ void control_warp(GroupSmem<NP, G> &sm, const ModalArgs &A, unsigned 
     }
 }
 
-// ------------------------------------------------------------------ compute warps
-// The stream of TMA chunks of one compute warp: per group iteration, 8 chunks
-// of x1/x2 for the A sweep, then 8 chunks of x1/x2/x3 for the C sweep.
+// ------------------------------------------------------------------ producer warp
+// Streams every compute warp's chunks with TMA: per group iteration, chunks
+// 0..7 carry x1/x2 rows of the unit for the A sweep, chunks 8..15 x1/x2/x3
+// rows for the C sweep.  Chunk q of warp w goes to buffer q % kRing once the
+// warp has released the chunk that used the buffer before.
 template <int NP, int G>
-struct ChunkStream {
-    static constexpr int kRing = GroupTraits<G>::kRing;
-    GroupSmem<NP, G> &sm;
-    const CUtensorMap *tm1, *tm2, *tm3;
-    const ModalArgs &A;
-    int w;
-    int issued;     // next chunk number to issue
-    int issue_gid;  // group id of the chunks being issued
-    int issue_k;    // group iteration of issue_gid
-
-    // Issues chunk number qn (lane 0).  Returns false at the end marker.
-    __device__ __forceinline__ bool issue_one(int qn)
-    {
+__device__ void producer_warp(GroupSmem<NP, G> &sm, const CUtensorMap *tm1, const CUtensorMap *tm2,
+                              const CUtensorMap *tm3, const ModalArgs &A)
+{
+    constexpr int kRing = GroupTraits<G>::kRing;
+    const int lane = threadIdx.x & 31;
+    int cur_k = -1;
+    GroupPos q{};
+    for (int qn = 0;; ++qn) {
         const int k = qn / kChunksPerGroup;
         const int c = qn % kChunksPerGroup;
-        if (k != issue_k) {
+        if (k != cur_k) {
             (void)mbar_wait_or_flag(&sm.gready[k & 1], (k >> 1) & 1, A.hdr);
-            issue_gid = sm.gid[k & 1];
-            issue_k = k;
+            const int gi = sm.gid[k & 1];
+            if (gi < 0) break;
+            q = group_pos(static_cast<unsigned int>(gi), A);
+            cur_k = k;
         }
-        if (issue_gid < 0) return false;
-        const GroupPos q = group_pos(static_cast<unsigned int>(issue_gid), A);
-        const int row = (static_cast<int>(q.s) * G + w) * MT + (c % kChunksPerSweep) * MCK;
         const int b = qn % kRing;
-        uint64_t *bar = &sm.full[w][b];
-        fence_proxy_async_smem();
-        if (c < kChunksPerSweep) {
-            mbar_arrive_expect_tx(bar, 2 * kChunkBytes);
-        } else {
-            mbar_arrive_expect_tx(bar, 3 * kChunkBytes);
-            tma_load_3d(sm.ring[w][b][2], tm3, bar, q.cb * MCH, row, q.b);
-        }
-        tma_load_3d(sm.ring[w][b][0], tm1, bar, q.cb * MCH, row, q.b);
-        tma_load_3d(sm.ring[w][b][1], tm2, bar, q.cb * MCH, row, q.b);
-        return true;
-    }
-
-    // Keeps the chunks up to number upto + kRing - 1 in flight (lane 0); the
-    // caller has finished reading chunk upto - 1.
-    __device__ __forceinline__ void top_up(int upto)
-    {
-        if ((threadIdx.x & 31) == 0) {
-            while (issued < upto + kRing) {
-                if (!issue_one(issued)) break;
-                ++issued;
+        const int row_in_unit = (c % kChunksPerSweep) * MCK;
+        for (int w = 0; w < G; ++w) {
+            if (qn >= kRing) (void)mbar_wait_or_flag(&sm.empty[w][b], ((qn / kRing) - 1) & 1, A.hdr);
+            if (lane == 0) {
+                const int row = (static_cast<int>(q.s) * G + w) * MT + row_in_unit;
+                uint64_t *bar = &sm.full[w][b];
+                fence_proxy_async_smem();
+                if (c < kChunksPerSweep) {
+                    mbar_arrive_expect_tx(bar, 2 * kChunkBytes);
+                } else {
+                    mbar_arrive_expect_tx(bar, 3 * kChunkBytes);
+                    tma_load_3d(sm.ring[w][b][2], tm3, bar, q.cb * MCH, row, q.b);
+                }
+                tma_load_3d(sm.ring[w][b][0], tm1, bar, q.cb * MCH, row, q.b);
+                tma_load_3d(sm.ring[w][b][1], tm2, bar, q.cb * MCH, row, q.b);
             }
         }
     }
-};
+}
 
+// ------------------------------------------------------------------ compute warps
 template <int NP>
 __device__ __forceinline__ void sweep_a_chunk(float2 (&s)[NP], const float2 (&p)[NP], const uint32_t *r1,
                                               const uint32_t *r2)
@@ -416,7 +412,7 @@ __device__ __forceinline__ void sweep_a_chunk(float2 (&s)[NP], const float2 (&p)
 }
 
 // One token of the C sweep for this lane's channel pair: advance the N states,
-// form conv = sum_n R_n s_n with four independent accumulation chains (all
+// form conv = sum_n R_n s_n with two independent accumulation chains (all
 // state updates first, so the chains find their inputs ready), apply the
 // gates and store y.
 template <int NP>
@@ -430,31 +426,26 @@ __device__ __forceinline__ void sweep_c_token(float2 (&s)[NP], const float2 (&p)
     for (int n = 0; n < NP; ++n) s[n] = __ffma2_rn(p[n], s[n], v);
     float2 a0 = __fmul2_rn(R[0], s[0]);
     float2 a1 = __fmul2_rn(R[1], s[1]);
-    float2 a2 = __fmul2_rn(R[2], s[2]);
-    float2 a3 = __fmul2_rn(R[3], s[3]);
 #pragma unroll
-    for (int n = 4; n < NP; n += 4) {
+    for (int n = 2; n < NP; n += 2) {
         a0 = __ffma2_rn(R[n], s[n], a0);
         a1 = __ffma2_rn(R[n + 1], s[n + 1], a1);
-        a2 = __ffma2_rn(R[n + 2], s[n + 2], a2);
-        a3 = __ffma2_rn(R[n + 3], s[n + 3], a3);
     }
-    const float2 conv = __fadd2_rn(__fadd2_rn(a0, a1), __fadd2_rn(a2, a3));
+    const float2 conv = __fadd2_rn(a0, a1);
     const float2 yv = __ffma2_rn(dsk, v, __fmul2_rn(x3, conv));
     st_pred_u32(yp, float2_to_bf16x2(yv), store);
 }
 
 template <int NP, int G>
-__device__ void compute_warp(GroupSmem<NP, G> &sm, const CUtensorMap *tm1, const CUtensorMap *tm2,
-                             const CUtensorMap *tm3, const ModalArgs &A)
+__device__ void compute_warp(GroupSmem<NP, G> &sm, const ModalArgs &A)
 {
     constexpr int kRing = GroupTraits<G>::kRing;
     const int lane = threadIdx.x & 31;
     const int w = threadIdx.x >> 5;
-    ChunkStream<NP, G> cs{sm, tm1, tm2, tm3, A, w, 0, -1, -1};
+    const int groups_per_chain = (A.units + G - 1) / G;
+    const size_t slot_floats = static_cast<size_t>(MGMAX + 1) * NP * MCH;
     int used = 0;  // next chunk number to consume
 
-    cs.top_up(0);
     for (int k = 0;; ++k) {
         (void)mbar_wait_or_flag(&sm.gready[k & 1], (k >> 1) & 1, A.hdr);
         const int gi = sm.gid[k & 1];
@@ -475,10 +466,22 @@ __device__ void compute_warp(GroupSmem<NP, G> &sm, const CUtensorMap *tm1, const
             (void)mbar_wait_tiles(&sm.full[w][b], (used / kRing) & 1, A.hdr);
             sweep_a_chunk<NP>(s, p, sm.ring[w][b][0] + lane, sm.ring[w][b][1] + lane);
             __syncwarp();
-            cs.top_up(used + 1);
+            if (lane == 0) mbar_arrive(&sm.empty[w][b]);
         }
 #pragma unroll
         for (int n = 0; n < NP; ++n) sm.ac[w][n * 32 + lane] = s[n];
+        // The aggregate also goes to the group's ring slot (for successors'
+        // look-backs); the fence lets the control warp release the flag
+        // without a fence of its own.
+        if (q.s > 0u && static_cast<int>(q.s) + 1 < groups_per_chain) {
+            const unsigned int chain = static_cast<unsigned int>(q.b) * A.nCB + q.cb;
+            float *slot = A.slots + (static_cast<size_t>(chain) * MRING + q.s % MRING) * slot_floats +
+                          static_cast<size_t>(w) * NP * MCH + 2 * lane;
+            (void)mbar_wait_or_flag(&sm.slotok[k & 1], (k >> 1) & 1, A.hdr);
+#pragma unroll
+            for (int n = 0; n < NP; ++n) *reinterpret_cast<float2 *>(slot + n * MCH) = s[n];
+            __threadfence();
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.adone[k & 1]);
 
@@ -499,18 +502,17 @@ __device__ void compute_warp(GroupSmem<NP, G> &sm, const CUtensorMap *tm1, const
             const uint32_t *r2 = sm.ring[w][b][1] + lane;
             const uint32_t *r3 = sm.ring[w][b][2] + lane;
             const int base = i * MCK;
+            uint32_t *yc = yrow + static_cast<size_t>(base) * ystride;
             if (base + MCK <= nvalid) {
 #pragma unroll
                 for (int r = 0; r < MCK; ++r)
-                    sweep_c_token<NP>(s, p, R, dsk, r1[r * 32], r2[r * 32], r3[r * 32],
-                                      yrow + static_cast<size_t>(base + r) * ystride, ch_ok);
+                    sweep_c_token<NP>(s, p, R, dsk, r1[r * 32], r2[r * 32], r3[r * 32], yc + r * ystride, ch_ok);
             } else {
                 for (int r = 0; r < MCK && base + r < nvalid; ++r)
-                    sweep_c_token<NP>(s, p, R, dsk, r1[r * 32], r2[r * 32], r3[r * 32],
-                                      yrow + static_cast<size_t>(base + r) * ystride, ch_ok);
+                    sweep_c_token<NP>(s, p, R, dsk, r1[r * 32], r2[r * 32], r3[r * 32], yc + r * ystride, ch_ok);
             }
             __syncwarp();
-            cs.top_up(used + 1);
+            if (lane == 0) mbar_arrive(&sm.empty[w][b]);
         }
         // A ragged last unit: the final state is the recurrence state after
         // token L-1 (its aggregate covers zero-padded rows).
@@ -540,9 +542,13 @@ __global__ void __launch_bounds__(GroupTraits<G>::kThreads, GroupTraits<G>::kCta
 
     if (threadIdx.x == 0) {
         for (int w = 0; w < G; ++w)
-            for (int b = 0; b < GroupTraits<G>::kRing; ++b) mbar_init(&sm.full[w][b], 1);
+            for (int b = 0; b < GroupTraits<G>::kRing; ++b) {
+                mbar_init(&sm.full[w][b], 1);
+                mbar_init(&sm.empty[w][b], 1);
+            }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.gready[i], 1);
+            mbar_init(&sm.slotok[i], 1);
             mbar_init(&sm.adone[i], G);
             mbar_init(&sm.cdone[i], 1);
         }
@@ -550,12 +556,16 @@ __global__ void __launch_bounds__(GroupTraits<G>::kThreads, GroupTraits<G>::kCta
     }
     __syncthreads();
 
-    if ((threadIdx.x >> 5) == G)
+    const int warp = threadIdx.x >> 5;
+    if (warp == G)
         control_warp<NP, G>(sm, A, epoch);
+    else if (warp == G + 1)
+        producer_warp<NP, G>(sm, &tm1, &tm2, &tm3, A);
     else
-        compute_warp<NP, G>(sm, &tm1, &tm2, &tm3, A);
+        compute_warp<NP, G>(sm, A);
 
-    // Every TMA a compute warp issued has been waited on by that warp.
+    // Every chunk the producer issued belongs to a group the compute warps
+    // consumed in full, so no TMA is in flight here.
     __syncthreads();
     // The last CTA to leave resets the ticket and advances the epoch so the
     // workspace is ready for the next launch without a memset.

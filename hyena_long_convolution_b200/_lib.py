@@ -37,6 +37,8 @@ SIGNATURES = {
     "hyena_modal_workspace_init": (_I, [_P, _SZ, _P]),
     "hyena_modal_long_conv": (_I, [_P, _P, _P, _I64, _P, _P, _P, _P, _I64, _P, _P,
                                    _I, _I, _I, _I, _P, _SZ, _P]),
+    "hyena_modal_long_conv_noalloc": (_I, [_P, _P, _P, _I64, _P, _P, _P, _P, _I64, _P, _P,
+                                           _I, _I, _I, _I, _P]),
     "hyena_modal_state_init": (_I, [_P, _I, _I, _I, _P]),
     "hyena_workspace_check": (_I, [_P, _P]),
 }

@@ -84,6 +84,8 @@ void record_cuda_error(cudaError_t e, const char *where)
     snprintf(g_last_error, sizeof g_last_error, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
+void record_message(const char *msg) { snprintf(g_last_error, sizeof g_last_error, "%s", msg); }
+
 ModalLayout modal_layout(int B, int D, int N)
 {
     ModalLayout L;

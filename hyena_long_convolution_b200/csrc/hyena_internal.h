@@ -14,6 +14,7 @@ namespace hyena {
 // Remembers the most recent failing CUDA call of this thread (reported by
 // hyena_last_error_message).
 void record_cuda_error(cudaError_t e, const char *where);
+void record_message(const char *msg);
 
 #define HYENA_TRY(call, where)                       \
     do {                                             \

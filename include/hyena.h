@@ -139,6 +139,40 @@ hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t 
                                      void *stream);
 
 /*
+ * Allocation-free variant of hyena_modal_long_conv (no counterpart on the
+ * pages: it exists for callers of this library that must not allocate device
+ * memory).  Some callers cannot call cudaMalloc or take memory from an
+ * allocator: a plugin that runs inside a host framework which owns all device
+ * memory and accounts for it, or code on a latency-critical path where an
+ * allocation could synchronise the device.  This entry point takes the same
+ * inputs and outputs as hyena_modal_long_conv but no workspace: its scratch
+ * is a fixed array of HYENA_NOALLOC_SCRATCH_BYTES in device memory that the
+ * library owns (every GPU that loads that part of the library holds it until
+ * the process exits).  It calls no allocating routine.
+ *
+ * Limit: B, D, N must satisfy
+ *   hyena_modal_long_conv_workspace_size(B, D, N) <= HYENA_NOALLOC_SCRATCH_BYTES
+ * (at N = 16: B * ceil(D / 64) <= 73 channel blocks, e.g. B = 1 and D up to
+ * 4672); larger sizes return HYENA_ERR_WORKSPACE and launch nothing.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the one array: calls that overlap on the GPU (on
+ * different streams, or from different threads without ordering) race and
+ * produce wrong results.  Each call clears the array's counters before its
+ * launch; a bounded-wait timeout inside the kernel invalidates that call's
+ * output and is not reported by this entry point.
+ */
+#define HYENA_NOALLOC_SCRATCH_BYTES (24u << 20)
+
+hyena_status_t hyena_modal_long_conv_noalloc(const hyena_bf16_t *x1, const hyena_bf16_t *x2,
+                                             const hyena_bf16_t *x3, int64_t ld_x,
+                                             const float *log_poles, const float *residues,
+                                             const float *Dskip,
+                                             hyena_bf16_t *y, int64_t ld_y,
+                                             const float *state_in, float *state_out,
+                                             int B, int L, int D, int N, void *stream);
+
+/*
  * Zero-fills a modal state [B, D, N] fp32 (the state before the first token
  * of a sequence): the start of chunked prefill.
  */

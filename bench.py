@@ -62,6 +62,35 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
+KERNEL_SOURCES = ("hyena_long_convolution_b200/csrc/modal_scan.cu",
+                  "hyena_long_convolution_b200/csrc/short_conv.cu",
+                  "hyena_long_convolution_b200/csrc/hyena_device.cuh",
+                  "hyena_long_convolution_b200/csrc/hyena_internal.h")
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, or None when the kernel sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(workload)
+    except Exception:
+        return None
+    if not rec or rec.get("kernel_sources_sha256_16") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -382,14 +411,7 @@ def run_gpu(args, wl):
     per_sorted = sorted(per)
     avg_ms = statistics.mean(per)
     achieved = BYTES_PER_CHTOK * chtok / (avg_ms / 1e3) / 1e9
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        try:
-            with open(tpath) as f:
-                traffic = json.load(f).get(args.workload)
-        except Exception:
-            traffic = None
+    traffic = recorded_traffic(args.workload)
 
     line = {
         "metric": METRIC,

@@ -197,8 +197,13 @@ __device__ void control_warp(GroupSmem<NP, G> &sm, const ModalArgs &A, unsigned 
     const size_t slot_floats = static_cast<size_t>(MGMAX + 1) * NP * MCH;
     const size_t incl_off = static_cast<size_t>(MGMAX) * NP * MCH;
 
+    // Tickets are taken one group ahead (so the producer can prefetch the next
+    // group's rows) when there are at least two groups per CTA; otherwise a
+    // CTA takes its next ticket only once its group is done, so that the
+    // groups spread over all CTAs instead of pairing up on half of them.
+    const int ahead = A.nGroups >= 2u * gridDim.x ? 2 : 1;
     announce_group<NP, G>(sm, A, 0);
-    announce_group<NP, G>(sm, A, 1);
+    if (ahead == 2) announce_group<NP, G>(sm, A, 1);
     for (int k = 0;; ++k) {
         __syncwarp();
         const int gi = sm.gid[k & 1];  // written by lane 0 of this warp
@@ -350,7 +355,7 @@ __device__ void control_warp(GroupSmem<NP, G> &sm, const ModalArgs &A, unsigned 
             if (lane == 0) st_release_u64(chain_flags + (s % MRING), flag_word(epoch, s, true));
         }
 
-        announce_group<NP, G>(sm, A, k + 2);
+        announce_group<NP, G>(sm, A, k + ahead);
     }
 }
 

@@ -9,13 +9,16 @@
 //
 // Design.  One CTA owns FCH = 64 channels x FT = 128 output tokens of one
 // batch row.  TMA stages x1, x2 for the tile plus a halo of HR >= K-1 earlier
-// rows (a second, shorter box) and x3 for the tile; v = x1 x2 is formed once in
-// fp32 into shared memory (halo rows before t = 0 come from hist_in).  Warp w
-// computes FRW = 16 consecutive outputs for the lane's two channels with a
-// register-blocked sliding window: per block of 8 taps it loads the 8 taps and
-// the 23 window values it needs and issues 8 x 16 packed f32x2 FMAs.  The
-// gates are applied in registers and y is stored as coalesced 128-byte rows.
-// A second small kernel writes hist_out (the last K-1 values of v).
+// rows (a second, shorter box) and x3 for the tile.  The bf16 x1 and x2 rows
+// land inside the fp32 buffer that then holds v = x1 x2 (two bf16 rows take
+// the bytes of one fp32 row), and are converted in place through registers
+// (halo rows before t = 0 come from hist_in), which keeps the CTA small
+// enough for two per SM even at K = 128.  Warp w computes FRW = 16
+// consecutive outputs for the lane's two channels with a register-blocked
+// sliding window: per block of 8 taps it loads the 8 taps and the 23 window
+// values it needs and issues 8 x 16 packed f32x2 FMAs.  The gates are applied
+// in registers and y is stored as coalesced 128-byte rows.  A second small
+// kernel writes hist_out (the last K-1 values of v).
 #include "hyena_device.cuh"
 #include "hyena_internal.h"
 
@@ -27,28 +30,43 @@ constexpr int kMaxHalo = 128;  // HR <= 128 since K <= 128
 constexpr int kRowWords = FCH / 2;  // 32-bit words per bf16 row
 
 struct FirSmemView {
-    uint32_t *x1, *x2, *x3;  // [HR + FT][32], [HR + FT][32], [FT][32]
+    uint32_t *x1, *x2, *x3;  // bf16 rows [HR + FT][32], [HR + FT][32], [FT][32]
     float2 *v;               // [HR + FT][32]
     float2 *taps;            // [K][32]
     uint64_t *bar;
 };
 
-__host__ __device__ inline size_t fir_smem_bytes(int HR, int K)
+// kInPlace: the bf16 x1, x2 rows land inside v's buffer (two bf16 rows take
+// the bytes of one fp32 row) instead of in buffers of their own.
+__host__ __device__ inline size_t fir_smem_bytes(int HR, int K, bool kInPlace)
 {
     const size_t rows = static_cast<size_t>(HR) + FT;
-    return rows * kRowWords * 4 * 2 + static_cast<size_t>(FT) * kRowWords * 4 + rows * 32 * 8 +
-           static_cast<size_t>(K) * 32 * 8 + 16;
+    const size_t raw = kInPlace ? 0 : rows * kRowWords * 4 * 2;
+    return raw + rows * 32 * 8 + static_cast<size_t>(FT) * kRowWords * 4 + static_cast<size_t>(K) * 32 * 8 + 16;
 }
 
+// The in-place layout is used when the separate one would not let two CTAs
+// share an SM (long filters, with their long halos).
+__host__ inline bool fir_in_place(int HR, int K) { return fir_smem_bytes(HR, K, false) > 112u * 1024u; }
+
+template <bool kInPlace>
 __device__ inline FirSmemView fir_smem(unsigned char *base, int HR, int K)
 {
     FirSmemView s;
     const int rows = HR + FT;
-    s.x1 = reinterpret_cast<uint32_t *>(base);
-    s.x2 = s.x1 + rows * kRowWords;
-    s.x3 = s.x2 + rows * kRowWords;
-    s.v = reinterpret_cast<float2 *>(s.x3 + FT * kRowWords);
-    s.taps = s.v + rows * 32;
+    if (kInPlace) {
+        s.v = reinterpret_cast<float2 *>(base);
+        s.x1 = reinterpret_cast<uint32_t *>(base);  // first half of v's bytes
+        s.x2 = s.x1 + rows * kRowWords;               // second half
+        s.x3 = reinterpret_cast<uint32_t *>(s.v + rows * 32);
+        s.taps = reinterpret_cast<float2 *>(s.x3 + FT * kRowWords);
+    } else {
+        s.x1 = reinterpret_cast<uint32_t *>(base);
+        s.x2 = s.x1 + rows * kRowWords;
+        s.x3 = s.x2 + rows * kRowWords;
+        s.v = reinterpret_cast<float2 *>(s.x3 + FT * kRowWords);
+        s.taps = s.v + rows * 32;
+    }
     s.bar = reinterpret_cast<uint64_t *>(s.taps + K * 32);
     return s;
 }
@@ -71,6 +89,7 @@ __device__ __forceinline__ void fir_block(float2 (&acc)[FRW], const float2 *vbas
         for (int i = 0; i < FRW; ++i) acc[i] = __ffma2_rn(tq[q], w[i - q + NQ - 1], acc[i]);
 }
 
+template <bool kInPlace>
 __global__ void __launch_bounds__(FW * 32)
     fir_kernel(const __grid_constant__ CUtensorMap tm1, const __grid_constant__ CUtensorMap tm2,
                const __grid_constant__ CUtensorMap tm3, const __grid_constant__ CUtensorMap th1,
@@ -79,7 +98,7 @@ __global__ void __launch_bounds__(FW * 32)
     extern __shared__ __align__(128) unsigned char smem_raw[];
     const int HR = A.HR;
     const int K = A.K;
-    FirSmemView sm = fir_smem(smem_raw, HR, K);
+    FirSmemView sm = fir_smem<kInPlace>(smem_raw, HR, K);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int cb = blockIdx.x;
     const int t0 = blockIdx.y * FT;
@@ -104,15 +123,36 @@ __global__ void __launch_bounds__(FW * 32)
         tma_load_3d(sm.x3, &tm3, sm.bar, cb * FCH, t0, b);
     }
     // taps -> fp32 [K][lane] while the tiles are in flight
-    for (int idx = tid; idx < K * 32; idx += FW * 32) {
-        const int k = idx >> 5, l = idx & 31;
-        const int c = cb * FCH + 2 * l;
-        float2 t = make_float2(0.f, 0.f);
-        if (c < A.D) {
-            t.x = __uint_as_float(static_cast<uint32_t>(A.taps[static_cast<size_t>(c) * K + k]) << 16);
-            t.y = __uint_as_float(static_cast<uint32_t>(A.taps[static_cast<size_t>(c + 1) * K + k]) << 16);
+    if ((K & 7) == 0) {
+        // 8 consecutive taps of one channel per 16-byte load
+        for (int idx = tid; idx < (K / 8) * 32; idx += FW * 32) {
+            const int l = idx & 31, kb = (idx >> 5) * 8;
+            const int c = cb * FCH + 2 * l;
+            uint4 ta = make_uint4(0u, 0u, 0u, 0u), tb = ta;
+            if (c < A.D) {
+                ta = __ldg(reinterpret_cast<const uint4 *>(A.taps + static_cast<size_t>(c) * K + kb));
+                tb = __ldg(reinterpret_cast<const uint4 *>(A.taps + static_cast<size_t>(c + 1) * K + kb));
+            }
+            const uint32_t wa[4] = {ta.x, ta.y, ta.z, ta.w}, wb[4] = {tb.x, tb.y, tb.z, tb.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 lo = make_float2(__uint_as_float(wa[i] << 16), __uint_as_float(wb[i] << 16));
+                const float2 hi = make_float2(__uint_as_float(wa[i] & 0xffff0000u), __uint_as_float(wb[i] & 0xffff0000u));
+                sm.taps[(kb + 2 * i) * 32 + l] = lo;
+                sm.taps[(kb + 2 * i + 1) * 32 + l] = hi;
+            }
         }
-        sm.taps[idx] = t;
+    } else {
+        for (int idx = tid; idx < K * 32; idx += FW * 32) {
+            const int k = idx >> 5, l = idx & 31;
+            const int c = cb * FCH + 2 * l;
+            float2 t = make_float2(0.f, 0.f);
+            if (c < A.D) {
+                t.x = __uint_as_float(static_cast<uint32_t>(A.taps[static_cast<size_t>(c) * K + k]) << 16);
+                t.y = __uint_as_float(static_cast<uint32_t>(A.taps[static_cast<size_t>(c + 1) * K + k]) << 16);
+            }
+            sm.taps[idx] = t;
+        }
     }
     const bool ok = mbar_wait_bounded(sm.bar, 0);
     if (__syncthreads_or(!ok)) {
@@ -121,20 +161,37 @@ __global__ void __launch_bounds__(FW * 32)
     }
 
     // v = x1 * x2 for the halo and the tile; rows before t = 0 from hist_in.
+    // In place, every thread first reads the bf16 words of its rows and then,
+    // after the barrier, writes their fp32 products over them.
     const int H = K - 1;
-    for (int r = warp; r < HR + FT; r += FW) {
+    const int rows = HR + FT;
+    auto v_of = [&](int r, uint32_t a, uint32_t bw) {
         const int t = t0 - HR + r;
-        float2 v;
-        if (t >= 0) {
-            v = __fmul2_rn(bf16x2_to_float2(sm.x1[r * kRowWords + lane]),
-                           bf16x2_to_float2(sm.x2[r * kRowWords + lane]));
-        } else if (t >= -H && A.hist_in != nullptr && ch_ok) {
-            const float *h = A.hist_in + (static_cast<size_t>(b) * H + (H + t)) * A.D + c0;
-            v = *reinterpret_cast<const float2 *>(h);
-        } else {
-            v = make_float2(0.f, 0.f);
+        if (t >= 0) return __fmul2_rn(bf16x2_to_float2(a), bf16x2_to_float2(bw));
+        if (t >= -H && A.hist_in != nullptr && ch_ok)
+            return *reinterpret_cast<const float2 *>(A.hist_in + (static_cast<size_t>(b) * H + (H + t)) * A.D + c0);
+        return make_float2(0.f, 0.f);
+    };
+    if constexpr (kInPlace) {
+        constexpr int kMaxRowsPerWarp = (kMaxHalo + FT) / FW;
+        uint32_t w1[kMaxRowsPerWarp], w2[kMaxRowsPerWarp];
+#pragma unroll
+        for (int i = 0; i < kMaxRowsPerWarp; ++i) {
+            const int r = warp + i * FW;
+            if (r < rows) {
+                w1[i] = sm.x1[r * kRowWords + lane];
+                w2[i] = sm.x2[r * kRowWords + lane];
+            }
         }
-        sm.v[r * 32 + lane] = v;
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < kMaxRowsPerWarp; ++i) {
+            const int r = warp + i * FW;
+            if (r < rows) sm.v[r * 32 + lane] = v_of(r, w1[i], w2[i]);
+        }
+    } else {
+        for (int r = warp; r < rows; r += FW)
+            sm.v[r * 32 + lane] = v_of(r, sm.x1[r * kRowWords + lane], sm.x2[r * kRowWords + lane]);
     }
     __syncthreads();
 
@@ -208,21 +265,26 @@ int launch_fir(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &
 {
     int launches = 0;
     if (a.L > 0) {
-        const size_t smem = fir_smem_bytes(a.HR, a.K);
-        static size_t configured = 0;
+        const bool in_place = fir_in_place(a.HR, a.K);
+        const size_t smem = fir_smem_bytes(a.HR, a.K, in_place);
         static int configured_device = -1;
         int dev = 0;
         HYENA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
-        if (configured_device != dev || smem > configured) {
-            const size_t max_smem = fir_smem_bytes(kMaxHalo, HYENA_MAX_TAPS);
-            HYENA_TRY(cudaFuncSetAttribute(fir_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(max_smem)),
+        if (configured_device != dev) {
+            // the largest request of either layout (halos up to kMaxHalo rows)
+            HYENA_TRY(cudaFuncSetAttribute(fir_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(fir_smem_bytes(kMaxHalo, HYENA_MAX_TAPS, true))),
                       "fir: set max dynamic shared memory");
-            configured = max_smem;
+            HYENA_TRY(cudaFuncSetAttribute(fir_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(fir_smem_bytes(kMaxHalo, HYENA_MAX_TAPS, false))),
+                      "fir: set max dynamic shared memory");
             configured_device = dev;
         }
         const dim3 grid((a.D + FCH - 1) / FCH, (a.L + FT - 1) / FT, a.B);
-        fir_kernel<<<grid, FW * 32, smem, st>>>(m1, m2, m3, h1, h2, a);
+        if (in_place)
+            fir_kernel<true><<<grid, FW * 32, smem, st>>>(m1, m2, m3, h1, h2, a);
+        else
+            fir_kernel<false><<<grid, FW * 32, smem, st>>>(m1, m2, m3, h1, h2, a);
         HYENA_TRY(cudaGetLastError(), "fir launch");
         ++launches;
     }

@@ -197,13 +197,13 @@ __device__ void control_warp(GroupSmem<NP, G> &sm, const ModalArgs &A, unsigned 
     const size_t slot_floats = static_cast<size_t>(MGMAX + 1) * NP * MCH;
     const size_t incl_off = static_cast<size_t>(MGMAX) * NP * MCH;
 
-    // Tickets are taken one group ahead (so the producer can prefetch the next
-    // group's rows) when there are at least two groups per CTA; otherwise a
-    // CTA takes its next ticket only once its group is done, so that the
-    // groups spread over all CTAs instead of pairing up on half of them.
-    const int ahead = A.nGroups >= 2u * gridDim.x ? 2 : 1;
+    // A CTA takes its next ticket when it has formed the carries of its
+    // current group: early enough for the producer to prefetch the next
+    // group's rows during the current output sweep, late enough that groups
+    // start in about ticket order (a look-back then rarely waits on a group
+    // that started late) and that short sequences spread over all CTAs.
+    constexpr int ahead = 1;
     announce_group<NP, G>(sm, A, 0);
-    if (ahead == 2) announce_group<NP, G>(sm, A, 1);
     for (int k = 0;; ++k) {
         __syncwarp();
         const int gi = sm.gid[k & 1];  // written by lane 0 of this warp

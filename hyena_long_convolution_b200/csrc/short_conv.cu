@@ -15,8 +15,9 @@
 // (halo rows before t = 0 come from hist_in), which keeps the CTA small
 // enough for two per SM even at K = 128.  Warp w computes FRW = 16
 // consecutive outputs for the lane's two channels with a register-blocked
-// sliding window: per block of 8 taps it loads the 8 taps and the 23 window
-// values it needs and issues 8 x 16 packed f32x2 FMAs.  The gates are applied
+// window: per block of 8 taps it issues 8 x 16 packed f32x2 FMAs on the 8 taps
+// and 23 window values, 15 of them carried over in registers from the
+// previous block (the window slides along the taps).  The gates are applied
 // in registers and y is stored as coalesced 128-byte rows.  A second small
 // kernel writes hist_out (the last K-1 values of v).
 #include "hyena_device.cuh"
@@ -87,6 +88,40 @@ __device__ __forceinline__ void fir_block(float2 (&acc)[FRW], const float2 *vbas
     for (int q = 0; q < NQ; ++q)
 #pragma unroll
         for (int i = 0; i < FRW; ++i) acc[i] = __ffma2_rn(tq[q], w[i - q + NQ - 1], acc[i]);
+}
+
+// Taps [0, 8*nblk) in blocks of 8 with the window sliding along the taps in
+// registers: block kb uses v rows [row0 - kb - 7, row0 - kb + 15]; the next
+// block reuses 15 of those 23 values and loads 8, which halves the
+// shared-memory traffic per FMA.  NBLK > 0: the block count is a compile-time
+// constant and the window shift is register renaming; NBLK == 0: runtime
+// count, the shift is register moves.
+template <int NBLK>
+__device__ __forceinline__ void fir_sliding8(float2 (&acc)[FRW], const float2 *v, const float2 *taps, int row0,
+                                             int nblk, int lane)
+{
+    constexpr int NW = FRW + 7;
+    if (NBLK > 0) nblk = NBLK;
+    float2 w[NW];
+#pragma unroll
+    for (int j = 0; j < NW; ++j) w[j] = v[(row0 - 7 + j) * 32 + lane];
+#pragma unroll(NBLK > 0 ? NBLK : 1)
+    for (int bk = 0; bk < nblk; ++bk) {
+        const int kb = bk * 8;
+        float2 tq[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) tq[q] = taps[(kb + q) * 32 + lane];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+#pragma unroll
+            for (int i = 0; i < FRW; ++i) acc[i] = __ffma2_rn(tq[q], w[i - q + 7], acc[i]);
+        if (bk + 1 < nblk) {
+#pragma unroll
+            for (int j = NW - 1; j >= 8; --j) w[j] = w[j - 8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) w[j] = v[(row0 - kb - 15 + j) * 32 + lane];
+        }
+    }
 }
 
 template <bool kInPlace>
@@ -199,9 +234,12 @@ __global__ void __launch_bounds__(FW * 32)
 #pragma unroll
     for (int i = 0; i < FRW; ++i) acc[i] = make_float2(0.f, 0.f);
     const int row0 = HR + warp * FRW;  // v row of this warp's first output
-    int kb = 0;
-    for (; kb + 8 <= K; kb += 8)
-        fir_block<8>(acc, sm.v + (row0 - kb - 7) * 32, sm.taps + kb * 32, lane);
+    const int nblk = K / 8;
+    if (nblk == HYENA_MAX_TAPS / 8)
+        fir_sliding8<HYENA_MAX_TAPS / 8>(acc, sm.v, sm.taps, row0, nblk, lane);
+    else if (nblk > 0)
+        fir_sliding8<0>(acc, sm.v, sm.taps, row0, nblk, lane);
+    const int kb = nblk * 8;
     switch (K - kb) {
         case 7: fir_block<7>(acc, sm.v + (row0 - kb - 6) * 32, sm.taps + kb * 32, lane); break;
         case 6: fir_block<6>(acc, sm.v + (row0 - kb - 5) * 32, sm.taps + kb * 32, lane); break;

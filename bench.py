@@ -82,16 +82,21 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
-KERNEL_SOURCES = ("hyena_long_convolution_b200/csrc/modal_scan.cu",
-                  "hyena_long_convolution_b200/csrc/short_conv.cu",
-                  "hyena_long_convolution_b200/csrc/hyena_device.cuh",
-                  "hyena_long_convolution_b200/csrc/hyena_internal.h")
+KERNEL_SOURCES = {
+    "modal": ("hyena_long_convolution_b200/csrc/modal_scan.cu",
+              "hyena_long_convolution_b200/csrc/hyena_device.cuh",
+              "hyena_long_convolution_b200/csrc/hyena_internal.h"),
+    "fir": ("hyena_long_convolution_b200/csrc/short_conv.cu",
+            "hyena_long_convolution_b200/csrc/hyena_device.cuh",
+            "hyena_long_convolution_b200/csrc/hyena_internal.h"),
+}
 
 
-def kernel_source_hash():
+def kernel_source_hash(kind="modal"):
+    """sha256/16 of the sources of one kernel family (modal scan or FIR)."""
     import hashlib
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kind]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -106,7 +111,7 @@ def recorded_traffic(workload):
             rec = json.load(f).get(workload)
     except Exception:
         return None
-    if not rec or rec.get("kernel_sources_sha256_16") != kernel_source_hash():
+    if not rec or rec.get("kernel_sources_sha256_16") != kernel_source_hash(WORKLOADS[workload]["kind"]):
         return None
     return rec.get("dram_bytes_per_launch")
 

@@ -49,6 +49,13 @@ WORKLOADS = {
                  desc="hcs explicit FIR K=7, B=2 L=8192 D=4096"),
     "fir128": dict(kind="fir", B=2, L=8192, D=4096, K=128, seed=1,
                    desc="hcm explicit FIR K=128, B=2 L=8192 D=4096"),
+    # generation: one step = L one-token decode calls (state / window carried)
+    "decode_modal": dict(kind="modal", decode=True, B=1, L=256, D=4096, N=16, seed=5, chunk=None,
+                         desc="hcl decode, B=1 D=4096 N=16, 256 one-token steps"),
+    "decode_modal_b64": dict(kind="modal", decode=True, B=64, L=64, D=4096, N=16, seed=6, chunk=None,
+                             desc="hcl decode, B=64 D=4096 N=16, 64 one-token steps"),
+    "decode_fir128": dict(kind="fir", decode=True, B=1, L=256, D=4096, K=128, seed=7,
+                          desc="hcm decode, B=1 D=4096 K=128, 256 one-token steps"),
 }
 
 
@@ -64,6 +71,20 @@ def alu_peak_tflops():
     except Exception:
         mhz = props.clock_rate / 1e3 if hasattr(props, "clock_rate") else 1965.0
     return props.multi_processor_count * 128 * 2 * mhz * 1e6 / 1e12
+
+
+def algorithmic_bytes(wl):
+    """Bytes a step must move at least: 8 per channel-token (x1, x2, x3 read,
+    y written) for prefill; a decode call also reads and writes the carried
+    state (N floats) or window (K-1 floats) and reads the filter parameters."""
+    chtok = wl["B"] * wl["L"] * wl["D"]
+    if not wl.get("decode"):
+        return BYTES_PER_CHTOK * chtok
+    if wl["kind"] == "modal":
+        per_call = wl["B"] * wl["D"] * (8 + 8 * wl["N"]) + wl["D"] * (8 * wl["N"] + 4)
+    else:
+        per_call = wl["B"] * wl["D"] * (8 + 8 * (wl["K"] - 1)) + wl["D"] * (2 * wl["K"] + 4)
+    return per_call * wl["L"]
 
 
 def flops_per_chtok(wl):
@@ -220,16 +241,19 @@ def oracle_sample_rate(wl, target_s=10.0):
         if wl["kind"] == "modal":
             inp = make_modal_inputs(B, L, D, wl["N"], wl["seed"], wl.get("wide", False))
             t = time.perf_counter()
-            if wl.get("chunk"):
+            if wl.get("chunk") or wl.get("decode"):
                 oracle.modal_chunked(inp["x1"], inp["x2"], inp["x3"], inp["log_poles"], inp["residues"],
-                                     inp["Dskip"], None, chunks=wl["chunk"])
+                                     inp["Dskip"], None, chunks=1 if wl.get("decode") else wl["chunk"])
             else:
                 oracle.modal_recurrence(inp["x1"], inp["x2"], inp["x3"], inp["log_poles"],
                                         inp["residues"], inp["Dskip"])
             return time.perf_counter() - t
         inp = make_fir_inputs(B, L, D, wl["K"], wl["seed"])
         t = time.perf_counter()
-        oracle.fir(inp["x1"], inp["x2"], inp["x3"], inp["taps"], None, None)
+        if wl.get("decode"):
+            oracle.fir_chunked(inp["x1"], inp["x2"], inp["x3"], inp["taps"], None, None, chunks=1)
+        else:
+            oracle.fir(inp["x1"], inp["x2"], inp["x3"], inp["taps"], None, None)
         return time.perf_counter() - t
 
     oracle.build()
@@ -287,6 +311,8 @@ class Step:
         if wl["kind"] == "modal":
             self.ws = hy.ModalWorkspace(B, D, wl["N"], device=device)
             self.S = torch.zeros((B, D, wl["N"]), device=device)
+        elif wl.get("decode"):
+            self.H = torch.zeros((B, wl["K"] - 1, D), device=device)
         self.graph = None
         if graph:
             s = torch.cuda.Stream(device=device)
@@ -303,6 +329,24 @@ class Step:
     def _run(self):
         hy, wl, d = self.hy, self.wl, self.dev
         n = 0
+        if wl.get("decode"):
+            # a generation loop: the state / window starts empty, one call per token
+            if wl["kind"] == "modal":
+                hy.modal_state_init(self.S)
+            else:
+                self.H.zero_()
+            n += 1
+            for t in range(wl["L"]):
+                sl = slice(t, t + 1)
+                if wl["kind"] == "modal":
+                    hy.modal_decode(d["x1"][:, sl], d["x2"][:, sl], d["x3"][:, sl], d["a"], d["R"], d["Ds"], self.S,
+                                    y=self.y[:, sl])
+                else:
+                    hy.short_decode(d["x1"][:, sl], d["x2"][:, sl], d["x3"][:, sl], d["taps"], None, self.H,
+                                    y=self.y[:, sl])
+                n += hy.last_launch_count()
+            self.launches = n
+            return
         if wl["kind"] == "modal":
             if wl.get("chunk"):
                 hy.modal_state_init(self.S)
@@ -364,12 +408,25 @@ def e2e_leg(wl, host, dev, device, steps, warmup):
     y = torch.empty((B, L, D), dtype=torch.bfloat16, device=device)
     if wl["kind"] == "modal":
         ws = hy.ModalWorkspace(B, D, wl["N"], device=device)
+        S = torch.zeros((B, D, wl["N"]), device=device)
+    elif wl.get("decode"):
+        H = torch.zeros((B, wl["K"] - 1, D), device=device)
 
     def step():
         for k in hx:
             dx[k].copy_(hx[k], non_blocking=True)
         bf = {k: dx[k].view(torch.bfloat16) for k in ("x1", "x2", "x3")}
-        if wl["kind"] == "modal":
+        if wl.get("decode"):
+            (S.zero_() if wl["kind"] == "modal" else H.zero_())
+            for t in range(L):
+                sl = slice(t, t + 1)
+                if wl["kind"] == "modal":
+                    hy.modal_decode(bf["x1"][:, sl], bf["x2"][:, sl], bf["x3"][:, sl], dx["a"], dx["R"], dx["Ds"],
+                                    S, y=y[:, sl])
+                else:
+                    hy.short_decode(bf["x1"][:, sl], bf["x2"][:, sl], bf["x3"][:, sl],
+                                    dx["taps"].view(torch.bfloat16), None, H, y=y[:, sl])
+        elif wl["kind"] == "modal":
             hy.modal_long_conv(bf["x1"], bf["x2"], bf["x3"], dx["a"], dx["R"], dx["Ds"], y=y, workspace=ws)
         else:
             hy.short_conv(bf["x1"], bf["x2"], bf["x3"], dx["taps"].view(torch.bfloat16), None, y=y)
@@ -435,13 +492,14 @@ def run_gpu(args, wl):
     peak, peak_kind = measured_peaks()
     per_sorted = sorted(per)
     avg_ms = statistics.mean(per)
-    achieved = BYTES_PER_CHTOK * chtok / (avg_ms / 1e3) / 1e9
+    step_bytes = algorithmic_bytes(wl)
+    achieved = step_bytes / (avg_ms / 1e3) / 1e9
     traffic = recorded_traffic(args.workload)
     # The roofline that bounds the path: HBM (8 B per channel-token) unless
     # the algorithmic flops take longer at the SIMT peak (long explicit FIRs).
     alu_peak = alu_peak_tflops()
     flops = flops_per_chtok(wl) * chtok
-    if flops / (alu_peak * 1e12) > BYTES_PER_CHTOK * chtok / (peak * 1e9):
+    if flops / (alu_peak * 1e12) > step_bytes / (peak * 1e9):
         roof = {"bound": "alu", "achieved": flops / (avg_ms / 1e3) / 1e12, "peak": alu_peak, "unit": "TFLOP/s",
                 "peak_source": "derived: SMs x 128 FP32 lanes x 2 flops x max SM clock",
                 "algorithmic_flops_per_launch": flops}
@@ -449,7 +507,7 @@ def run_gpu(args, wl):
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "peak_source": f"{peak_kind} hbm_gbs (copy)"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof.update({"traffic": traffic, "algorithmic_bytes_per_launch": BYTES_PER_CHTOK * chtok,
+    roof.update({"traffic": traffic, "algorithmic_bytes_per_step": step_bytes,
                  "hbm_frac": achieved / peak, "kernel_ms_min": per_sorted[0], "kernel_ms_avg": avg_ms})
 
     line = {
@@ -468,6 +526,7 @@ def run_gpu(args, wl):
         "data": "synthetic (seeded N(0,1) bf16 inputs, pages' shapes)",
         "config": {"workload": wl["desc"], "B": wl["B"], "L": wl["L"], "D": wl["D"],
                    **({"N": wl["N"]} if wl["kind"] == "modal" else {"K": wl["K"]}),
+                   "mode": "decode (one-token calls)" if wl.get("decode") else "prefill",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "cache": "inputs larger than L2 (no flush)", "graph": bool(args.graph)},
         "roofline": roof,

@@ -23,9 +23,11 @@ __all__ = [
     "HyenaError",
     "ModalWorkspace",
     "last_launch_count",
+    "modal_decode",
     "modal_long_conv",
     "modal_state_init",
     "short_conv",
+    "short_decode",
     "workspace_check",
     "workspace_size",
 ]
@@ -156,6 +158,70 @@ def modal_long_conv(x1, x2, x3, log_poles, residues, Dskip=None, y=None, state_i
                                      _ptr(Dskip), _ptr(y), ld_y, _ptr(state_in), _ptr(state_out),
                                      B, L, D, N, _ptr(workspace.buf), workspace.nbytes, _stream(stream))
     check("hyena_modal_long_conv", rc)
+    return y
+
+
+def _bd(x, name):
+    """One token per batch row: [B, D] or [B, 1, D] bf16 with unit channel
+    stride -> (B, D, ld), element (b, c) at b * ld + c."""
+    torch = _torch()
+    if x.dtype != torch.bfloat16 or not x.is_cuda or x.dim() not in (2, 3) or (x.dim() == 3 and x.shape[1] != 1):
+        raise ValueError(f"{name} must be a bf16 CUDA tensor [B, D] or [B, 1, D]")
+    if x.stride(-1) != 1:
+        raise ValueError(f"{name} must have unit channel stride")
+    return x.shape[0], x.shape[-1], x.stride(0)
+
+
+def modal_decode(x1, x2, x3, log_poles, residues, Dskip, state, y=None, stream=None):
+    """One generated token through the long modal filter: advances ``state``
+    ([B, D, N] fp32, in place) and returns y ([B, D] or [B, 1, D] like x1).
+    Equals ``modal_long_conv`` on a one-token sequence with state_in =
+    state_out = state, bit for bit."""
+    torch = _torch()
+    (B, D, ld), b2, b3 = _bd(x1, "x1"), _bd(x2, "x2"), _bd(x3, "x3")
+    if b2 != (B, D, ld) or b3 != (B, D, ld):
+        raise ValueError("x1, x2, x3 must share shape and row stride")
+    Dn, N = log_poles.shape
+    if Dn != D:
+        raise ValueError("log_poles must be [D, N]")
+    _f32(log_poles, (D, N), "log_poles", False)
+    _f32(residues, (D, N), "residues", False)
+    _f32(Dskip, (D,), "Dskip")
+    _f32(state, (B, D, N), "state", False)
+    if y is None:
+        y = torch.empty_like(x1, memory_format=torch.contiguous_format)
+    yB, yD, ld_y = _bd(y, "y")
+    if (yB, yD) != (B, D):
+        raise ValueError("y shape differs from x")
+    rc = lib().hyena_modal_decode(_ptr(x1), _ptr(x2), _ptr(x3), ld, _ptr(log_poles), _ptr(residues), _ptr(Dskip),
+                                  _ptr(y), ld_y, _ptr(state), B, D, N, _stream(stream))
+    check("hyena_modal_decode", rc)
+    return y
+
+
+def short_decode(x1, x2, x3, taps, Dskip, hist, y=None, stream=None):
+    """One generated token through an explicit FIR: advances the window
+    ``hist`` ([B, K-1, D] fp32, in place; None when K = 1) and returns y.
+    Equals ``short_conv`` on a one-token sequence with hist_in = hist_out =
+    hist, bit for bit."""
+    torch = _torch()
+    (B, D, ld), b2, b3 = _bd(x1, "x1"), _bd(x2, "x2"), _bd(x3, "x3")
+    if b2 != (B, D, ld) or b3 != (B, D, ld):
+        raise ValueError("x1, x2, x3 must share shape and row stride")
+    if taps.dtype != torch.bfloat16 or taps.dim() != 2 or taps.shape[0] != D or not taps.is_contiguous():
+        raise ValueError("taps must be a contiguous bf16 [D, K] tensor")
+    K = taps.shape[1]
+    _f32(Dskip, (D,), "Dskip")
+    if K > 1:
+        _f32(hist, (B, K - 1, D), "hist", False)
+    if y is None:
+        y = torch.empty_like(x1, memory_format=torch.contiguous_format)
+    yB, yD, ld_y = _bd(y, "y")
+    if (yB, yD) != (B, D):
+        raise ValueError("y shape differs from x")
+    rc = lib().hyena_short_decode(_ptr(x1), _ptr(x2), _ptr(x3), ld, _ptr(taps), _ptr(Dskip), _ptr(y), ld_y,
+                                  _ptr(hist) if K > 1 else None, B, D, K, _stream(stream))
+    check("hyena_short_decode", rc)
     return y
 
 

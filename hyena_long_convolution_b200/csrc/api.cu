@@ -270,6 +270,64 @@ hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t 
     return HYENA_OK;
 }
 
+hyena_status_t hyena_modal_decode(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
+                                  int64_t ld_x, const float *log_poles, const float *residues, const float *Dskip,
+                                  hyena_bf16_t *y, int64_t ld_y, float *state, int B, int D, int N, void *stream)
+{
+    hyena_status_t st = check_x(x1, x2, x3, ld_x, y, ld_y, B, 1, D);
+    if (st != HYENA_OK) return st;
+    if (N < 1 || N > HYENA_MAX_MODES) return N < 1 ? HYENA_ERR_INVALID_ARG : HYENA_ERR_UNSUPPORTED;
+    if (!log_poles || !residues || !state) return HYENA_ERR_INVALID_ARG;
+    if (!aligned16(log_poles) || !aligned16(residues) || !aligned16(state) || (Dskip && !aligned16(Dskip)))
+        return HYENA_ERR_ALIGNMENT;
+    DecodeArgs a{};
+    a.x1 = x1;
+    a.x2 = x2;
+    a.x3 = x3;
+    a.ld_x = ld_x;
+    a.log_poles = log_poles;
+    a.residues = residues;
+    a.Dskip = Dskip;
+    a.y = y;
+    a.ld_y = ld_y;
+    a.state = state;
+    a.B = B;
+    a.D = D;
+    a.N = N;
+    const int n = launch_modal_decode(a, static_cast<cudaStream_t>(stream));
+    if (n < 0) return HYENA_ERR_CUDA;
+    g_last_launches = n;
+    return HYENA_OK;
+}
+
+hyena_status_t hyena_short_decode(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
+                                  int64_t ld_x, const hyena_bf16_t *taps, const float *Dskip, hyena_bf16_t *y,
+                                  int64_t ld_y, float *hist, int B, int D, int K, void *stream)
+{
+    hyena_status_t st = check_x(x1, x2, x3, ld_x, y, ld_y, B, 1, D);
+    if (st != HYENA_OK) return st;
+    if (K < 1 || K > HYENA_MAX_TAPS) return K < 1 ? HYENA_ERR_INVALID_ARG : HYENA_ERR_UNSUPPORTED;
+    if (taps == nullptr || (K > 1 && hist == nullptr)) return HYENA_ERR_INVALID_ARG;
+    if (!aligned16(taps) || (Dskip && !aligned16(Dskip)) || (K > 1 && !aligned16(hist))) return HYENA_ERR_ALIGNMENT;
+    DecodeArgs a{};
+    a.x1 = x1;
+    a.x2 = x2;
+    a.x3 = x3;
+    a.ld_x = ld_x;
+    a.taps = taps;
+    a.Dskip = Dskip;
+    a.y = y;
+    a.ld_y = ld_y;
+    a.hist = K > 1 ? hist : nullptr;
+    a.B = B;
+    a.D = D;
+    a.K = K;
+    const int n = launch_fir_decode(a, static_cast<cudaStream_t>(stream));
+    if (n < 0) return HYENA_ERR_CUDA;
+    g_last_launches = n;
+    return HYENA_OK;
+}
+
 hyena_status_t hyena_modal_state_init(float *state, int B, int D, int N, void *stream)
 {
     if (state == nullptr || B < 1 || D < 1 || N < 1) return HYENA_ERR_INVALID_ARG;

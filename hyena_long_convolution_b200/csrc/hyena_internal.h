@@ -100,6 +100,23 @@ struct FirArgs {
     float *hist_out;
 };
 
+// One-token decode step (modal state or FIR window advanced in place).
+struct DecodeArgs {
+    const uint16_t *x1, *x2, *x3;
+    long long ld_x;
+    const float *log_poles, *residues;  // modal
+    const uint16_t *taps;               // FIR
+    const float *Dskip;
+    uint16_t *y;
+    long long ld_y;
+    float *state;  // modal [B, D, N]
+    float *hist;   // FIR [B, K-1, D]
+    int B, D, N, K;
+};
+
+int launch_modal_decode(const DecodeArgs &a, cudaStream_t st);
+int launch_fir_decode(const DecodeArgs &a, cudaStream_t st);
+
 int launch_fir(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3,
                const CUtensorMap &h1, const CUtensorMap &h2, const FirArgs &a,
                cudaStream_t st);

@@ -173,6 +173,47 @@ hyena_status_t hyena_modal_long_conv_noalloc(const hyena_bf16_t *x1, const hyena
                                              int B, int L, int D, int N, void *stream);
 
 /*
+ * One generated token through the long modal filter: the recurrent form of
+ * hcl (Evo2-7B-262K model card, §Implementation Notes and "Custom cache":
+ * generation carries the IIR state from token to token).
+ *
+ *   v = x1 * x2;  s_n <- exp(log_poles[c,n]) * s_n + v;
+ *   y = x3 * sum_n residues[c,n] * s_n + Dskip[c] * v
+ *
+ * x1, x2, x3, y  one token per batch row: element (b, c) at b * ld + c.
+ * state  [B, D, N] fp32, device, read and updated in place: the state after
+ *        the previous token (zeros before the first one).  Required.
+ * log_poles, residues [D, N], Dskip [D] or NULL: as hyena_modal_long_conv.
+ * The result equals hyena_modal_long_conv with L = 1 and
+ * state_in = state_out = state bit for bit.  No workspace; one launch.
+ */
+hyena_status_t hyena_modal_decode(const hyena_bf16_t *x1, const hyena_bf16_t *x2,
+                                  const hyena_bf16_t *x3, int64_t ld_x,
+                                  const float *log_poles, const float *residues,
+                                  const float *Dskip,
+                                  hyena_bf16_t *y, int64_t ld_y,
+                                  float *state, int B, int D, int N, void *stream);
+
+/*
+ * One generated token through an explicit FIR (hcs/hcm): conv = sum_{k<K}
+ * taps[c,k] v[t-k] with v[t-k], k >= 1, from the window, which then advances
+ * by one token in place (Evo2-7B-262K model card, "Custom cache"; the FIR
+ * window of Evo1-1.5-7B-8K model card, "Cache subclass").
+ *
+ * hist   [B, K-1, D] fp32, device, in time order (hist[b, K-2, c] is v of the
+ *        previous token; zeros before the first one); read and updated in
+ *        place.  Required when K > 1, ignored when K = 1.
+ * taps   [D, K] bf16 in lag order, Dskip [D] or NULL: as hyena_short_conv.
+ * The result equals hyena_short_conv with L = 1 and hist_in = hist_out = hist
+ * bit for bit.  One launch.
+ */
+hyena_status_t hyena_short_decode(const hyena_bf16_t *x1, const hyena_bf16_t *x2,
+                                  const hyena_bf16_t *x3, int64_t ld_x,
+                                  const hyena_bf16_t *taps, const float *Dskip,
+                                  hyena_bf16_t *y, int64_t ld_y,
+                                  float *hist, int B, int D, int K, void *stream);
+
+/*
  * Zero-fills a modal state [B, D, N] fp32 (the state before the first token
  * of a sequence): the start of chunked prefill.
  */

@@ -100,6 +100,31 @@ def test_short_conv_rejects_bad_arguments(kw, code):
     assert fir(hy.lib(), **kw) == code
 
 
+def mdec(lib, x1=A, x2=A, x3=A, ld_x=64, a=A, R=A, Ds=None, y=A, ld_y=64, state=A, B=1, D=64, N=8):
+    return lib.hyena_modal_decode(x1, x2, x3, ld_x, a, R, Ds, y, ld_y, state, B, D, N, None)
+
+
+def fdec(lib, x1=A, x2=A, x3=A, ld_x=64, taps=A, Ds=None, y=A, ld_y=64, hist=A, B=1, D=64, K=7):
+    return lib.hyena_short_decode(x1, x2, x3, ld_x, taps, Ds, y, ld_y, hist, B, D, K, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), INVALID), (dict(state=None), INVALID), (dict(a=None), INVALID), (dict(R=None), INVALID),
+    (dict(y=None), INVALID), (dict(N=0), INVALID), (dict(N=17), UNSUP), (dict(ld_x=32), INVALID),
+    (dict(state=A + 4), ALIGN), (dict(x2=A + 2), ALIGN), (dict(Ds=A + 8), ALIGN), (dict(D=12, ld_x=16, ld_y=16), ALIGN),
+])
+def test_modal_decode_rejects_bad_arguments(kw, code):
+    assert mdec(hy.lib(), **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), INVALID), (dict(taps=None), INVALID), (dict(hist=None), INVALID), (dict(K=0), INVALID),
+    (dict(K=129), UNSUP), (dict(hist=A + 4), ALIGN), (dict(taps=A + 2), ALIGN), (dict(ld_y=16), INVALID),
+])
+def test_short_decode_rejects_bad_arguments(kw, code):
+    assert fdec(hy.lib(), **kw) == code
+
+
 def test_other_entry_points_reject_bad_arguments():
     lib = hy.lib()
     assert lib.hyena_modal_state_init(None, 1, 64, 8, None) == INVALID

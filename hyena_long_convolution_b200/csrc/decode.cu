@@ -32,8 +32,29 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits(float f)
     return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
+constexpr int kDecodeThreads = 64;  // small blocks: more CTAs (SMs) per call at batch 1
+
+// N consecutive floats at p (16-byte aligned when N % 4 == 0) into v[0, N).
 template <int NP>
-__global__ void __launch_bounds__(256) modal_decode_kernel(const DecodeArgs A)
+__device__ __forceinline__ void load_row(float (&v)[NP], const float *p, int N)
+{
+    if (N == NP) {
+#pragma unroll
+        for (int i = 0; i < NP; i += 4) {
+            const float4 q = __ldg(reinterpret_cast<const float4 *>(p + i));
+            v[i] = q.x;
+            v[i + 1] = q.y;
+            v[i + 2] = q.z;
+            v[i + 3] = q.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < NP; ++i) v[i] = i < N ? p[i] : 0.f;
+    }
+}
+
+template <int NP>
+__global__ void __launch_bounds__(kDecodeThreads) modal_decode_kernel(const DecodeArgs A)
 {
     const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (idx >= static_cast<long long>(A.B) * A.D) return;
@@ -42,19 +63,27 @@ __global__ void __launch_bounds__(256) modal_decode_kernel(const DecodeArgs A)
     const size_t xi = static_cast<size_t>(b) * A.ld_x + c;
     const float v = __fmul_rn(bf16_bits_to_float(A.x1[xi]), bf16_bits_to_float(A.x2[xi]));
     const float x3 = bf16_bits_to_float(A.x3[xi]);
-    const float *a = A.log_poles + static_cast<size_t>(c) * A.N;
-    const float *R = A.residues + static_cast<size_t>(c) * A.N;
     float *st = A.state + (static_cast<size_t>(b) * A.D + c) * A.N;
 
-    float s[NP], r[NP];
+    // padded modes (n >= N): p = R = 0 and a zero state, as in the prefill kernel
+    float a[NP], r[NP], s[NP];
+    load_row<NP>(a, A.log_poles + static_cast<size_t>(c) * A.N, A.N);
+    load_row<NP>(r, A.residues + static_cast<size_t>(c) * A.N, A.N);
+    if (A.N == NP) {
 #pragma unroll
-    for (int n = 0; n < NP; ++n) {
-        // padded modes: p = R = 0 and a zero state, as in the prefill kernel
-        const bool real = n < A.N;
-        const float p = real ? expf(a[n]) : 0.f;
-        r[n] = real ? R[n] : 0.f;
-        s[n] = __fmaf_rn(p, real ? st[n] : 0.f, v);
+        for (int i = 0; i < NP; i += 4) {
+            const float4 q = *reinterpret_cast<const float4 *>(st + i);
+            s[i] = q.x;
+            s[i + 1] = q.y;
+            s[i + 2] = q.z;
+            s[i + 3] = q.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < NP; ++i) s[i] = i < A.N ? st[i] : 0.f;
     }
+#pragma unroll
+    for (int n = 0; n < NP; ++n) s[n] = __fmaf_rn(n < A.N ? expf(a[n]) : 0.f, s[n], v);
     float a0 = __fmul_rn(r[0], s[0]);
     float a1 = __fmul_rn(r[1], s[1]);
 #pragma unroll
@@ -65,13 +94,23 @@ __global__ void __launch_bounds__(256) modal_decode_kernel(const DecodeArgs A)
     const float conv = __fadd_rn(a0, a1);
     const float dsk = A.Dskip != nullptr ? A.Dskip[c] : 0.f;
     A.y[static_cast<size_t>(b) * A.ld_y + c] = float_to_bf16_bits(__fmaf_rn(dsk, v, __fmul_rn(x3, conv)));
+    if (A.N == NP) {
 #pragma unroll
-    for (int n = 0; n < NP; ++n)
-        if (n < A.N) st[n] = s[n];
+        for (int i = 0; i < NP; i += 4)
+            *reinterpret_cast<float4 *>(st + i) = make_float4(s[i], s[i + 1], s[i + 2], s[i + 3]);
+    } else {
+#pragma unroll
+        for (int n = 0; n < NP; ++n)
+            if (n < A.N) st[n] = s[n];
+    }
 }
 
 // hist [B, K-1, D] in time order: hist[b][K-2][c] is v of the previous token.
-__global__ void __launch_bounds__(256) fir_decode_kernel(const DecodeArgs A)
+// One pass from the newest window entry to the oldest: each entry is read
+// once, feeds the lag-ordered FMA chain (lag k = K-1-j for entry j) and is
+// written one place older, through a carry register, so the window advances
+// in place.
+__global__ void __launch_bounds__(kDecodeThreads) fir_decode_kernel(const DecodeArgs A)
 {
     const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (idx >= static_cast<long long>(A.B) * A.D) return;
@@ -82,17 +121,38 @@ __global__ void __launch_bounds__(256) fir_decode_kernel(const DecodeArgs A)
     const float v = __fmul_rn(bf16_bits_to_float(A.x1[xi]), bf16_bits_to_float(A.x2[xi]));
     const float x3 = bf16_bits_to_float(A.x3[xi]);
     const uint16_t *tp = A.taps + static_cast<size_t>(c) * K;
-    float *hist = A.hist + static_cast<size_t>(b) * H * A.D + c;  // element j at hist[j * D]
+    const size_t D = static_cast<size_t>(A.D);
+    float *hist = A.hist + static_cast<size_t>(b) * H * D + c;  // entry j at hist[j * D]
 
-    // taps in lag order, from an accumulator starting at +0 (as the prefill
-    // kernel's register accumulators do)
+    // lag 0, from an accumulator starting at +0 (as the prefill kernel's
+    // register accumulators do)
     float acc = __fmaf_rn(bf16_bits_to_float(tp[0]), v, 0.f);
-    for (int k = 1; k < K; ++k) acc = __fmaf_rn(bf16_bits_to_float(tp[k]), hist[static_cast<size_t>(H - k) * A.D], acc);
+    float carry = v;  // the value entry j receives
+    // Entries in batches of 32 (lags k0 .. k0+31, entries H-k0 down): all of a
+    // batch's loads are issued before its FMAs and stores.
+    constexpr int kBatch = 32;
+    for (int k0 = 1; k0 < K; k0 += kBatch) {
+        float old[kBatch], tap[kBatch];
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+            const int k = k0 + i;
+            if (k < K) {
+                old[i] = hist[static_cast<size_t>(H - k) * D];
+                tap[i] = bf16_bits_to_float(tp[k]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+            const int k = k0 + i;
+            if (k < K) {
+                acc = __fmaf_rn(tap[i], old[i], acc);
+                hist[static_cast<size_t>(H - k) * D] = carry;
+                carry = old[i];
+            }
+        }
+    }
     const float dsk = A.Dskip != nullptr ? A.Dskip[c] : 0.f;
     A.y[static_cast<size_t>(b) * A.ld_y + c] = float_to_bf16_bits(__fmaf_rn(dsk, v, __fmul_rn(x3, acc)));
-    // advance the window: each thread owns its channel's column, read before written
-    for (int j = 0; j + 1 < H; ++j) hist[static_cast<size_t>(j) * A.D] = hist[static_cast<size_t>(j + 1) * A.D];
-    if (H > 0) hist[static_cast<size_t>(H - 1) * A.D] = v;
 }
 
 }  // namespace
@@ -100,11 +160,11 @@ __global__ void __launch_bounds__(256) fir_decode_kernel(const DecodeArgs A)
 int launch_modal_decode(const DecodeArgs &a, cudaStream_t st)
 {
     const long long n = static_cast<long long>(a.B) * a.D;
-    const unsigned int grid = static_cast<unsigned int>((n + 255) / 256);
+    const unsigned int grid = static_cast<unsigned int>((n + kDecodeThreads - 1) / kDecodeThreads);
     switch (modal_padded_modes(a.N)) {
-        case 4: modal_decode_kernel<4><<<grid, 256, 0, st>>>(a); break;
-        case 8: modal_decode_kernel<8><<<grid, 256, 0, st>>>(a); break;
-        default: modal_decode_kernel<16><<<grid, 256, 0, st>>>(a); break;
+        case 4: modal_decode_kernel<4><<<grid, kDecodeThreads, 0, st>>>(a); break;
+        case 8: modal_decode_kernel<8><<<grid, kDecodeThreads, 0, st>>>(a); break;
+        default: modal_decode_kernel<16><<<grid, kDecodeThreads, 0, st>>>(a); break;
     }
     HYENA_TRY(cudaGetLastError(), "modal decode launch");
     return 1;
@@ -113,7 +173,8 @@ int launch_modal_decode(const DecodeArgs &a, cudaStream_t st)
 int launch_fir_decode(const DecodeArgs &a, cudaStream_t st)
 {
     const long long n = static_cast<long long>(a.B) * a.D;
-    fir_decode_kernel<<<static_cast<unsigned int>((n + 255) / 256), 256, 0, st>>>(a);
+    fir_decode_kernel<<<static_cast<unsigned int>((n + kDecodeThreads - 1) / kDecodeThreads), kDecodeThreads, 0,
+                        st>>>(a);
     HYENA_TRY(cudaGetLastError(), "fir decode launch");
     return 1;
 }

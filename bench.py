@@ -49,6 +49,15 @@ WORKLOADS = {
                  desc="hcs explicit FIR K=7, B=2 L=8192 D=4096"),
     "fir128": dict(kind="fir", B=2, L=8192, D=4096, K=128, seed=1,
                    desc="hcm explicit FIR K=128, B=2 L=8192 D=4096"),
+    # inputs read from one projection buffer interleaved per channel triple
+    # (x1_c, x2_c, x3_c adjacent), the in_proj output layout
+    "modal32k_triples": dict(kind="modal", B=1, L=32768, D=4096, N=16, seed=2, chunk=None, group=1,
+                             desc="hcl modal long conv, B=1 L=32768 D=4096 N=16, single pass, "
+                                  "inputs interleaved per channel triple"),
+    "fir7_triples": dict(kind="fir", B=2, L=8192, D=4096, K=7, seed=1, group=1,
+                         desc="hcs explicit FIR K=7, B=2 L=8192 D=4096, inputs interleaved per channel triple"),
+    "fir128_triples": dict(kind="fir", B=2, L=8192, D=4096, K=128, seed=1, group=1,
+                           desc="hcm explicit FIR K=128, B=2 L=8192 D=4096, inputs interleaved per channel triple"),
     # generation: one step = L one-token decode calls (state / window carried)
     "decode_modal": dict(kind="modal", decode=True, B=1, L=256, D=4096, N=16, seed=5, chunk=None,
                          desc="hcl decode, B=1 D=4096 N=16, 256 one-token steps"),
@@ -293,6 +302,15 @@ def make_device_inputs(wl, device):
         inp = make_fir_inputs(wl["B"], wl["L"], wl["D"], wl["K"], wl["seed"])
         host = dict(x1=inp["x1"], x2=inp["x2"], x3=inp["x3"], taps=inp["taps"])
         dev = dict(x1=up(inp["x1"]), x2=up(inp["x2"]), x3=up(inp["x3"]), taps=up(inp["taps"]))
+    if wl.get("group"):
+        # one [B, L, 3D] projection buffer, channel groups of `group` as [x1 | x2 | x3]
+        G = wl["group"]
+        B, L, D = wl["B"], wl["L"], wl["D"]
+        xp = np.stack([host.pop(k).reshape(B, L, D // G, G) for k in ("x1", "x2", "x3")], axis=3)
+        host["xp"] = np.ascontiguousarray(xp.reshape(B, L, 3 * D))
+        for k in ("x1", "x2", "x3"):
+            del dev[k]
+        dev["xp"] = up(host["xp"])
     return host, dev
 
 
@@ -346,6 +364,14 @@ class Step:
                                     y=self.y[:, sl])
                 n += hy.last_launch_count()
             self.launches = n
+            return
+        if wl.get("group"):
+            if wl["kind"] == "modal":
+                hy.modal_long_conv_packed(d["xp"], wl["group"], d["a"], d["R"], d["Ds"], y=self.y,
+                                          state_out=self.S, workspace=self.ws)
+            else:
+                hy.short_conv_packed(d["xp"], wl["group"], d["taps"], None, y=self.y)
+            self.launches = hy.last_launch_count()
             return
         if wl["kind"] == "modal":
             if wl.get("chunk"):
@@ -415,8 +441,13 @@ def e2e_leg(wl, host, dev, device, steps, warmup):
     def step():
         for k in hx:
             dx[k].copy_(hx[k], non_blocking=True)
-        bf = {k: dx[k].view(torch.bfloat16) for k in ("x1", "x2", "x3")}
-        if wl.get("decode"):
+        bf = {k: dx[k].view(torch.bfloat16) for k in ("x1", "x2", "x3", "xp") if k in dx}
+        if wl.get("group"):
+            if wl["kind"] == "modal":
+                hy.modal_long_conv_packed(bf["xp"], wl["group"], dx["a"], dx["R"], dx["Ds"], y=y, workspace=ws)
+            else:
+                hy.short_conv_packed(bf["xp"], wl["group"], dx["taps"].view(torch.bfloat16), None, y=y)
+        elif wl.get("decode"):
             (S.zero_() if wl["kind"] == "modal" else H.zero_())
             for t in range(L):
                 sl = slice(t, t + 1)
@@ -527,6 +558,8 @@ def run_gpu(args, wl):
         "config": {"workload": wl["desc"], "B": wl["B"], "L": wl["L"], "D": wl["D"],
                    **({"N": wl["N"]} if wl["kind"] == "modal" else {"K": wl["K"]}),
                    "mode": "decode (one-token calls)" if wl.get("decode") else "prefill",
+                   "input_layout": (f"packed projection, channel groups of {wl['group']}" if wl.get("group")
+                                    else "three [B, L, D] tensors"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "cache": "inputs larger than L2 (no flush)", "graph": bool(args.graph)},
         "roofline": roof,

@@ -11,7 +11,9 @@ with h_c either an explicit short FIR (hcs 7 taps / hcm 128 taps,
 ``short_conv``) or the long modal filter h_c[t] = sum_n R[c,n] exp(a[c,n] t)
 (hcl, ``modal_long_conv``).  Layout [B, L, D] bf16, channel-contiguous; a row
 stride ld >= D is allowed, so x1, x2, x3 may be views of one [B, L, 3D]
-projection output.
+projection output.  The ``*_packed`` variants read the three inputs from one
+[B, L, >= 3D] projection buffer whose rows hold channel groups of ``group``
+channels as [x1 | x2 | x3] (group = 1: per-channel triples x1_c x2_c x3_c).
 """
 from __future__ import annotations
 
@@ -24,10 +26,14 @@ __all__ = [
     "ModalWorkspace",
     "last_launch_count",
     "modal_decode",
+    "modal_decode_packed",
     "modal_long_conv",
+    "modal_long_conv_packed",
     "modal_state_init",
     "short_conv",
+    "short_conv_packed",
     "short_decode",
+    "short_decode_packed",
     "workspace_check",
     "workspace_size",
 ]
@@ -251,4 +257,114 @@ def short_conv(x1, x2, x3, taps, Dskip=None, y=None, hist_in=None, hist_out=None
     rc = lib().hyena_short_conv(_ptr(x1), _ptr(x2), _ptr(x3), ld, _ptr(taps), _ptr(Dskip), _ptr(y), ld_y,
                                 _ptr(hist_in), _ptr(hist_out), B, L, D, K, _stream(stream))
     check("hyena_short_conv", rc)
+    return y
+
+
+# ---------------------------------------------------------------- packed inputs
+
+def _packed(xp, D, decode=False):
+    """Projection buffer [B, L, W] (decode: [B, W] or [B, 1, W]) with W >= 3D
+    and unit element stride -> (B, L, ld)."""
+    if decode:
+        B, W, ld = _bd(xp, "xp")
+        L = 1
+    else:
+        B, L, W, ld = _bld(xp, "xp")
+    if W < 3 * D:
+        raise ValueError(f"xp rows hold {W} values, fewer than 3 D = {3 * D}")
+    return B, L, ld
+
+
+def modal_long_conv_packed(xp, group, log_poles, residues, Dskip=None, y=None, state_in=None,
+                           state_out=None, workspace: ModalWorkspace | None = None, stream=None):
+    """``modal_long_conv`` with x1, x2, x3 read from one projection buffer xp
+    ([B, L, W >= 3D] bf16) in channel groups of ``group`` (x_k of channel c at
+    column 3 group (c // group) + (k-1) group + c % group).  D is taken from
+    log_poles ([D, N])."""
+    torch = _torch()
+    D, N = log_poles.shape
+    B, L, ld = _packed(xp, D)
+    _f32(log_poles, (D, N), "log_poles", False)
+    _f32(residues, (D, N), "residues", False)
+    _f32(Dskip, (D,), "Dskip")
+    _f32(state_in, (B, D, N), "state_in")
+    _f32(state_out, (B, D, N), "state_out")
+    if y is None:
+        y = torch.empty((B, L, D), dtype=torch.bfloat16, device=xp.device)
+    yB, yL, yD, ld_y = _bld(y, "y")
+    if (yB, yL, yD) != (B, L, D):
+        raise ValueError("y must be [B, L, D]")
+    if workspace is None:
+        workspace = ModalWorkspace(B, D, N, device=xp.device, stream=stream)
+    rc = lib().hyena_modal_long_conv_packed(_ptr(xp), ld, int(group), _ptr(log_poles), _ptr(residues),
+                                            _ptr(Dskip), _ptr(y), ld_y, _ptr(state_in), _ptr(state_out),
+                                            B, L, D, N, _ptr(workspace.buf), workspace.nbytes, _stream(stream))
+    check("hyena_modal_long_conv_packed", rc)
+    return y
+
+
+def short_conv_packed(xp, group, taps, Dskip=None, y=None, hist_in=None, hist_out=None, stream=None):
+    """``short_conv`` with x1, x2, x3 read from one projection buffer xp in
+    channel groups of ``group`` (see ``modal_long_conv_packed``).  D is taken
+    from taps ([D, K])."""
+    torch = _torch()
+    if taps.dtype != torch.bfloat16 or taps.dim() != 2 or not taps.is_contiguous():
+        raise ValueError("taps must be a contiguous bf16 [D, K] tensor")
+    D, K = taps.shape
+    B, L, ld = _packed(xp, D)
+    _f32(Dskip, (D,), "Dskip")
+    _f32(hist_in, (B, K - 1, D), "hist_in")
+    _f32(hist_out, (B, K - 1, D), "hist_out")
+    if y is None:
+        y = torch.empty((B, L, D), dtype=torch.bfloat16, device=xp.device)
+    yB, yL, yD, ld_y = _bld(y, "y")
+    if (yB, yL, yD) != (B, L, D):
+        raise ValueError("y must be [B, L, D]")
+    rc = lib().hyena_short_conv_packed(_ptr(xp), ld, int(group), _ptr(taps), _ptr(Dskip), _ptr(y), ld_y,
+                                       _ptr(hist_in), _ptr(hist_out), B, L, D, K, _stream(stream))
+    check("hyena_short_conv_packed", rc)
+    return y
+
+
+def modal_decode_packed(xp, group, log_poles, residues, Dskip, state, y=None, stream=None):
+    """``modal_decode`` with the token's x1, x2, x3 read from one projection
+    row per batch row (xp [B, W] or [B, 1, W], W >= 3D) in channel groups of
+    ``group``."""
+    torch = _torch()
+    D, N = log_poles.shape
+    B, _, ld = _packed(xp, D, decode=True)
+    _f32(log_poles, (D, N), "log_poles", False)
+    _f32(residues, (D, N), "residues", False)
+    _f32(Dskip, (D,), "Dskip")
+    _f32(state, (B, D, N), "state", False)
+    if y is None:
+        y = torch.empty((B, D), dtype=torch.bfloat16, device=xp.device)
+    yB, yD, ld_y = _bd(y, "y")
+    if (yB, yD) != (B, D):
+        raise ValueError("y must be [B, D] or [B, 1, D]")
+    rc = lib().hyena_modal_decode_packed(_ptr(xp), ld, int(group), _ptr(log_poles), _ptr(residues), _ptr(Dskip),
+                                         _ptr(y), ld_y, _ptr(state), B, D, N, _stream(stream))
+    check("hyena_modal_decode_packed", rc)
+    return y
+
+
+def short_decode_packed(xp, group, taps, Dskip, hist, y=None, stream=None):
+    """``short_decode`` with the token's x1, x2, x3 read from one projection
+    row per batch row in channel groups of ``group``."""
+    torch = _torch()
+    if taps.dtype != torch.bfloat16 or taps.dim() != 2 or not taps.is_contiguous():
+        raise ValueError("taps must be a contiguous bf16 [D, K] tensor")
+    D, K = taps.shape
+    B, _, ld = _packed(xp, D, decode=True)
+    _f32(Dskip, (D,), "Dskip")
+    if K > 1:
+        _f32(hist, (B, K - 1, D), "hist", False)
+    if y is None:
+        y = torch.empty((B, D), dtype=torch.bfloat16, device=xp.device)
+    yB, yD, ld_y = _bd(y, "y")
+    if (yB, yD) != (B, D):
+        raise ValueError("y must be [B, D] or [B, 1, D]")
+    rc = lib().hyena_short_decode_packed(_ptr(xp), ld, int(group), _ptr(taps), _ptr(Dskip), _ptr(y), ld_y,
+                                         _ptr(hist) if K > 1 else None, B, D, K, _stream(stream))
+    check("hyena_short_decode_packed", rc)
     return y

@@ -29,18 +29,63 @@ void resolve_encode()
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// 3-D bf16 tensor map over a [B, L, ld]-strided tensor, box [rows x 64 ch].
-bool encode_bf16_map(CUtensorMap *m, const void *base, int B, int L, int D, long long ld, int rows)
+// Where x1, x2, x3 are read from (see x_col): three tensors (group = D), a
+// packed projection buffer in channel groups, or per-channel triples.
+struct XSource {
+    const hyena_bf16_t *x[3];
+    long long ld;
+    int group;
+    bool triples;
+};
+
+XSource separate_source(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3, long long ld, int D)
+{
+    return XSource{{x1, x2, x3}, ld, D, false};
+}
+
+XSource packed_source(const hyena_bf16_t *xp, long long ld, int group)
+{
+    if (xp == nullptr) return XSource{{nullptr, nullptr, nullptr}, ld, group, group == 1};
+    return XSource{{xp, xp + group, xp + 2 * static_cast<long long>(group)}, ld, group, group == 1};
+}
+
+// 4-D bf16 tensor map [B][L][groups][group] over input k (0..2), box of `rows`
+// tokens x 64 channels: dims {group, D / group, L, B}, the group stride 3 group
+// elements (unused for a single group).  Triples: one map over the interleaved rows, dims {3D, 1, L, B},
+// box of `rows` tokens x 192 values (64 channels' triples).
+bool encode_x_map(CUtensorMap *m, const XSource &xs, int k, int B, int L, int D, int rows)
 {
     std::call_once(g_encode_once, resolve_encode);
     if (g_encode == nullptr) return false;
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
-                          static_cast<cuuint64_t>(B)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * 2,
-                             static_cast<cuuint64_t>(ld) * 2 * static_cast<cuuint64_t>(L)};
-    cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(rows), 1u};
-    cuuint32_t estr[3] = {1u, 1u, 1u};
-    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+    const cuuint64_t row_bytes = static_cast<cuuint64_t>(xs.ld) * 2;
+    cuuint64_t dims[4], strides[3];
+    cuuint32_t box[4];
+    if (xs.triples) {
+        dims[0] = 3ull * static_cast<cuuint64_t>(D);
+        dims[1] = 1;
+        strides[0] = row_bytes;
+        box[0] = 3u * 64u;
+        box[1] = 1u;
+    } else {
+        const int groups = D / xs.group;
+        dims[0] = static_cast<cuuint64_t>(xs.group);
+        dims[1] = static_cast<cuuint64_t>(groups);
+        strides[0] = groups > 1 ? 6ull * static_cast<cuuint64_t>(xs.group) : row_bytes;
+        // 64 channels per box: one run of 64 within a group (a single group
+        // reads past its end as zeros), or 64 / group whole groups of fewer
+        // than 64 channels (group divides 64)
+        const bool runs = groups == 1 || xs.group >= 64;
+        box[0] = static_cast<cuuint32_t>(runs ? 64 : xs.group);
+        box[1] = static_cast<cuuint32_t>(runs ? 1 : 64 / xs.group);
+    }
+    dims[2] = static_cast<cuuint64_t>(L);
+    dims[3] = static_cast<cuuint64_t>(B);
+    strides[1] = row_bytes;
+    strides[2] = row_bytes * static_cast<cuuint64_t>(L);
+    box[2] = static_cast<cuuint32_t>(rows);
+    box[3] = 1u;
+    cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<hyena_bf16_t *>(xs.x[k]), dims,
                                 strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                                 CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -63,6 +108,25 @@ hyena_status_t check_x(const void *x1, const void *x2, const void *x3, long long
         if (static_cast<long long>(L) * ld_x * 2 >= (1ll << 40)) return HYENA_ERR_UNSUPPORTED;
     }
     if (D % 8) return HYENA_ERR_ALIGNMENT;
+    return HYENA_OK;
+}
+
+// Checks of a packed projection buffer (the counterpart of check_x).
+hyena_status_t check_packed(const void *xp, long long ld_x, int group, const void *y, long long ld_y, int B, int L,
+                            int D)
+{
+    if (B < 1 || L < 0 || D < 1) return HYENA_ERR_INVALID_ARG;
+    if (D % 8) return HYENA_ERR_ALIGNMENT;
+    if (group < 1 || D % group) return HYENA_ERR_INVALID_ARG;
+    if (!(group == 1 || group == D || (group % 8 == 0 && (64 % group == 0 || group % 64 == 0))))
+        return HYENA_ERR_UNSUPPORTED;
+    if (L > 0) {
+        if (!xp || !y) return HYENA_ERR_INVALID_ARG;
+        if (ld_x < 3ll * D || ld_y < D) return HYENA_ERR_INVALID_ARG;
+        if ((ld_x % 8) || (ld_y % 8)) return HYENA_ERR_ALIGNMENT;
+        if (!aligned16(xp) || !aligned16(y)) return HYENA_ERR_ALIGNMENT;
+        if (static_cast<long long>(L) * ld_x * 2 >= (1ll << 40)) return HYENA_ERR_UNSUPPORTED;
+    }
     return HYENA_OK;
 }
 
@@ -111,35 +175,13 @@ ModalLayout modal_layout(int B, int D, int N)
 
 using namespace hyena;
 
-extern "C" {
+namespace {
 
-const char *hyena_status_string(hyena_status_t s)
+hyena_status_t short_conv_impl(const XSource &xs, const hyena_bf16_t *taps, const float *Dskip, hyena_bf16_t *y,
+                               int64_t ld_y, const float *hist_in, float *hist_out, int B, int L, int D, int K,
+                               void *stream)
 {
-    switch (s) {
-        case HYENA_OK: return "HYENA_OK";
-        case HYENA_ERR_INVALID_ARG: return "HYENA_ERR_INVALID_ARG";
-        case HYENA_ERR_ALIGNMENT: return "HYENA_ERR_ALIGNMENT";
-        case HYENA_ERR_UNSUPPORTED: return "HYENA_ERR_UNSUPPORTED";
-        case HYENA_ERR_CUDA: return "HYENA_ERR_CUDA";
-        case HYENA_ERR_TIMEOUT: return "HYENA_ERR_TIMEOUT";
-        case HYENA_ERR_WORKSPACE: return "HYENA_ERR_WORKSPACE";
-        default: return "HYENA_ERR_UNKNOWN";
-    }
-}
-
-int hyena_abi_version(void) { return 100; }
-
-int hyena_last_launch_count(void) { return g_last_launches; }
-
-const char *hyena_last_error_message(void) { return g_last_error; }
-
-hyena_status_t hyena_short_conv(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
-                                int64_t ld_x, const hyena_bf16_t *taps, const float *Dskip,
-                                hyena_bf16_t *y, int64_t ld_y, const float *hist_in, float *hist_out,
-                                int B, int L, int D, int K, void *stream)
-{
-    hyena_status_t st = check_x(x1, x2, x3, ld_x, y, ld_y, B, L, D);
-    if (st != HYENA_OK) return st;
+    hyena_status_t st = HYENA_OK;
     if (K < 1 || K > HYENA_MAX_TAPS) return K < 1 ? HYENA_ERR_INVALID_ARG : HYENA_ERR_UNSUPPORTED;
     if (taps == nullptr) return HYENA_ERR_INVALID_ARG;
     if ((Dskip && !aligned16(Dskip)) || (hist_in && !aligned16(hist_in)) ||
@@ -167,50 +209,40 @@ hyena_status_t hyena_short_conv(const hyena_bf16_t *x1, const hyena_bf16_t *x2, 
     a.D = D;
     a.K = K;
     a.HR = fir_halo_rows(K);
-    a.x1 = x1;
-    a.x2 = x2;
-    a.ld_x = ld_x;
+    a.x1 = xs.x[0];
+    a.x2 = xs.x[1];
+    a.ld_x = xs.ld;
+    a.group = xs.group;
     a.hist_out = hist_out;
     CUtensorMap m1, m2, m3, h1, h2;
-    if (!encode_bf16_map(&m1, x1, B, L, D, ld_x, FT) || !encode_bf16_map(&m2, x2, B, L, D, ld_x, FT) ||
-        !encode_bf16_map(&m3, x3, B, L, D, ld_x, FT))
+    if (!encode_x_map(&m1, xs, 0, B, L, D, FT)) return HYENA_ERR_CUDA;
+    if (xs.triples) {
+        m2 = m3 = m1;
+    } else if (!encode_x_map(&m2, xs, 1, B, L, D, FT) || !encode_x_map(&m3, xs, 2, B, L, D, FT)) {
         return HYENA_ERR_CUDA;
+    }
     if (a.HR > 0) {
-        if (!encode_bf16_map(&h1, x1, B, L, D, ld_x, a.HR) || !encode_bf16_map(&h2, x2, B, L, D, ld_x, a.HR))
+        if (!encode_x_map(&h1, xs, 0, B, L, D, a.HR)) return HYENA_ERR_CUDA;
+        if (xs.triples)
+            h2 = h1;
+        else if (!encode_x_map(&h2, xs, 1, B, L, D, a.HR))
             return HYENA_ERR_CUDA;
     } else {
         h1 = m1;
         h2 = m2;
     }
-    const int n = launch_fir(m1, m2, m3, h1, h2, a, s);
+    const int n = launch_fir(m1, m2, m3, h1, h2, a, xs.triples, s);
     if (n < 0) return HYENA_ERR_CUDA;
     g_last_launches = n;
     return HYENA_OK;
 }
 
-size_t hyena_modal_long_conv_workspace_size(int B, int D, int N)
+hyena_status_t modal_long_conv_impl(const XSource &xs, const float *log_poles, const float *residues,
+                                   const float *Dskip, hyena_bf16_t *y, int64_t ld_y, const float *state_in,
+                                   float *state_out, int B, int L, int D, int N, void *workspace,
+                                   size_t workspace_bytes, void *stream)
 {
-    if (B < 1 || D < 1 || N < 1 || N > HYENA_MAX_MODES) return 0;
-    return modal_layout(B, D, N).total;
-}
-
-hyena_status_t hyena_modal_workspace_init(void *workspace, size_t workspace_bytes, void *stream)
-{
-    if (workspace == nullptr || workspace_bytes == 0) return HYENA_ERR_INVALID_ARG;
-    if (cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return HYENA_ERR_CUDA;
-    g_last_launches = 1;
-    return HYENA_OK;
-}
-
-hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
-                                     int64_t ld_x, const float *log_poles, const float *residues,
-                                     const float *Dskip, hyena_bf16_t *y, int64_t ld_y,
-                                     const float *state_in, float *state_out, int B, int L, int D, int N,
-                                     void *workspace, size_t workspace_bytes, void *stream)
-{
-    hyena_status_t st = check_x(x1, x2, x3, ld_x, y, ld_y, B, L, D);
-    if (st != HYENA_OK) return st;
+    hyena_status_t st = HYENA_OK;
     if (N < 1) return HYENA_ERR_INVALID_ARG;
     if (N > HYENA_MAX_MODES) return HYENA_ERR_UNSUPPORTED;
     if (!log_poles || !residues) return HYENA_ERR_INVALID_ARG;
@@ -233,8 +265,9 @@ hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t 
 
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     ModalArgs a{};
-    a.x3 = x3;
-    a.ld_x = ld_x;
+    a.x3 = xs.x[2];
+    a.ld_x = xs.ld;
+    a.group = xs.group;
     a.y = y;
     a.ld_y = ld_y;
     a.state_in = state_in;
@@ -261,30 +294,31 @@ hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t 
     sy.coef = reinterpret_cast<float *>(ws + lay.off_coef);
 
     CUtensorMap m1, m2, m3;
-    if (!encode_bf16_map(&m1, x1, B, L, D, ld_x, MCK) || !encode_bf16_map(&m2, x2, B, L, D, ld_x, MCK) ||
-        !encode_bf16_map(&m3, x3, B, L, D, ld_x, MCK))
+    if (!encode_x_map(&m1, xs, 0, B, L, D, MCK)) return HYENA_ERR_CUDA;
+    if (xs.triples)
+        m2 = m3 = m1;
+    else if (!encode_x_map(&m2, xs, 1, B, L, D, MCK) || !encode_x_map(&m3, xs, 2, B, L, D, MCK))
         return HYENA_ERR_CUDA;
-    const int n = launch_modal(m1, m2, m3, a, sy, lay.NP, s);
+    const int n = launch_modal(m1, m2, m3, a, sy, lay.NP, xs.triples, s);
     if (n < 0) return HYENA_ERR_CUDA;
     g_last_launches = n;
     return HYENA_OK;
 }
 
-hyena_status_t hyena_modal_decode(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
-                                  int64_t ld_x, const float *log_poles, const float *residues, const float *Dskip,
-                                  hyena_bf16_t *y, int64_t ld_y, float *state, int B, int D, int N, void *stream)
+hyena_status_t modal_decode_impl(const XSource &xs, const float *log_poles, const float *residues,
+                                 const float *Dskip, hyena_bf16_t *y, int64_t ld_y, float *state, int B, int D, int N,
+                                 void *stream)
 {
-    hyena_status_t st = check_x(x1, x2, x3, ld_x, y, ld_y, B, 1, D);
-    if (st != HYENA_OK) return st;
     if (N < 1 || N > HYENA_MAX_MODES) return N < 1 ? HYENA_ERR_INVALID_ARG : HYENA_ERR_UNSUPPORTED;
     if (!log_poles || !residues || !state) return HYENA_ERR_INVALID_ARG;
     if (!aligned16(log_poles) || !aligned16(residues) || !aligned16(state) || (Dskip && !aligned16(Dskip)))
         return HYENA_ERR_ALIGNMENT;
     DecodeArgs a{};
-    a.x1 = x1;
-    a.x2 = x2;
-    a.x3 = x3;
-    a.ld_x = ld_x;
+    a.x1 = xs.x[0];
+    a.x2 = xs.x[1];
+    a.x3 = xs.x[2];
+    a.ld_x = xs.ld;
+    a.group = xs.group;
     a.log_poles = log_poles;
     a.residues = residues;
     a.Dskip = Dskip;
@@ -300,20 +334,18 @@ hyena_status_t hyena_modal_decode(const hyena_bf16_t *x1, const hyena_bf16_t *x2
     return HYENA_OK;
 }
 
-hyena_status_t hyena_short_decode(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
-                                  int64_t ld_x, const hyena_bf16_t *taps, const float *Dskip, hyena_bf16_t *y,
-                                  int64_t ld_y, float *hist, int B, int D, int K, void *stream)
+hyena_status_t short_decode_impl(const XSource &xs, const hyena_bf16_t *taps, const float *Dskip, hyena_bf16_t *y,
+                                 int64_t ld_y, float *hist, int B, int D, int K, void *stream)
 {
-    hyena_status_t st = check_x(x1, x2, x3, ld_x, y, ld_y, B, 1, D);
-    if (st != HYENA_OK) return st;
     if (K < 1 || K > HYENA_MAX_TAPS) return K < 1 ? HYENA_ERR_INVALID_ARG : HYENA_ERR_UNSUPPORTED;
     if (taps == nullptr || (K > 1 && hist == nullptr)) return HYENA_ERR_INVALID_ARG;
     if (!aligned16(taps) || (Dskip && !aligned16(Dskip)) || (K > 1 && !aligned16(hist))) return HYENA_ERR_ALIGNMENT;
     DecodeArgs a{};
-    a.x1 = x1;
-    a.x2 = x2;
-    a.x3 = x3;
-    a.ld_x = ld_x;
+    a.x1 = xs.x[0];
+    a.x2 = xs.x[1];
+    a.x3 = xs.x[2];
+    a.ld_x = xs.ld;
+    a.group = xs.group;
     a.taps = taps;
     a.Dskip = Dskip;
     a.y = y;
@@ -326,6 +358,127 @@ hyena_status_t hyena_short_decode(const hyena_bf16_t *x1, const hyena_bf16_t *x2
     if (n < 0) return HYENA_ERR_CUDA;
     g_last_launches = n;
     return HYENA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *hyena_status_string(hyena_status_t s)
+{
+    switch (s) {
+        case HYENA_OK: return "HYENA_OK";
+        case HYENA_ERR_INVALID_ARG: return "HYENA_ERR_INVALID_ARG";
+        case HYENA_ERR_ALIGNMENT: return "HYENA_ERR_ALIGNMENT";
+        case HYENA_ERR_UNSUPPORTED: return "HYENA_ERR_UNSUPPORTED";
+        case HYENA_ERR_CUDA: return "HYENA_ERR_CUDA";
+        case HYENA_ERR_TIMEOUT: return "HYENA_ERR_TIMEOUT";
+        case HYENA_ERR_WORKSPACE: return "HYENA_ERR_WORKSPACE";
+        default: return "HYENA_ERR_UNKNOWN";
+    }
+}
+
+int hyena_abi_version(void) { return 100; }
+
+int hyena_last_launch_count(void) { return g_last_launches; }
+
+const char *hyena_last_error_message(void) { return g_last_error; }
+
+size_t hyena_modal_long_conv_workspace_size(int B, int D, int N)
+{
+    if (B < 1 || D < 1 || N < 1 || N > HYENA_MAX_MODES) return 0;
+    return modal_layout(B, D, N).total;
+}
+
+hyena_status_t hyena_modal_workspace_init(void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (workspace == nullptr || workspace_bytes == 0) return HYENA_ERR_INVALID_ARG;
+    if (cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return HYENA_ERR_CUDA;
+    g_last_launches = 1;
+    return HYENA_OK;
+}
+
+hyena_status_t hyena_short_conv(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
+                                int64_t ld_x, const hyena_bf16_t *taps, const float *Dskip,
+                                hyena_bf16_t *y, int64_t ld_y, const float *hist_in, float *hist_out,
+                                int B, int L, int D, int K, void *stream)
+{
+    const hyena_status_t st = check_x(x1, x2, x3, ld_x, y, ld_y, B, L, D);
+    if (st != HYENA_OK) return st;
+    return short_conv_impl(separate_source(x1, x2, x3, ld_x, D), taps, Dskip, y, ld_y, hist_in, hist_out, B, L, D,
+                           K, stream);
+}
+
+hyena_status_t hyena_short_conv_packed(const hyena_bf16_t *xp, int64_t ld_x, int group, const hyena_bf16_t *taps,
+                                       const float *Dskip, hyena_bf16_t *y, int64_t ld_y, const float *hist_in,
+                                       float *hist_out, int B, int L, int D, int K, void *stream)
+{
+    const hyena_status_t st = check_packed(xp, ld_x, group, y, ld_y, B, L, D);
+    if (st != HYENA_OK) return st;
+    return short_conv_impl(packed_source(xp, ld_x, group), taps, Dskip, y, ld_y, hist_in, hist_out, B, L, D, K,
+                           stream);
+}
+
+hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
+                                     int64_t ld_x, const float *log_poles, const float *residues,
+                                     const float *Dskip, hyena_bf16_t *y, int64_t ld_y,
+                                     const float *state_in, float *state_out, int B, int L, int D, int N,
+                                     void *workspace, size_t workspace_bytes, void *stream)
+{
+    const hyena_status_t st = check_x(x1, x2, x3, ld_x, y, ld_y, B, L, D);
+    if (st != HYENA_OK) return st;
+    return modal_long_conv_impl(separate_source(x1, x2, x3, ld_x, D), log_poles, residues, Dskip, y, ld_y, state_in,
+                                state_out, B, L, D, N, workspace, workspace_bytes, stream);
+}
+
+hyena_status_t hyena_modal_long_conv_packed(const hyena_bf16_t *xp, int64_t ld_x, int group, const float *log_poles,
+                                            const float *residues, const float *Dskip, hyena_bf16_t *y,
+                                            int64_t ld_y, const float *state_in, float *state_out, int B, int L,
+                                            int D, int N, void *workspace, size_t workspace_bytes, void *stream)
+{
+    const hyena_status_t st = check_packed(xp, ld_x, group, y, ld_y, B, L, D);
+    if (st != HYENA_OK) return st;
+    return modal_long_conv_impl(packed_source(xp, ld_x, group), log_poles, residues, Dskip, y, ld_y, state_in,
+                                state_out, B, L, D, N, workspace, workspace_bytes, stream);
+}
+
+hyena_status_t hyena_modal_decode(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
+                                  int64_t ld_x, const float *log_poles, const float *residues, const float *Dskip,
+                                  hyena_bf16_t *y, int64_t ld_y, float *state, int B, int D, int N, void *stream)
+{
+    const hyena_status_t st = check_x(x1, x2, x3, ld_x, y, ld_y, B, 1, D);
+    if (st != HYENA_OK) return st;
+    return modal_decode_impl(separate_source(x1, x2, x3, ld_x, D), log_poles, residues, Dskip, y, ld_y, state, B, D,
+                             N, stream);
+}
+
+hyena_status_t hyena_modal_decode_packed(const hyena_bf16_t *xp, int64_t ld_x, int group, const float *log_poles,
+                                         const float *residues, const float *Dskip, hyena_bf16_t *y, int64_t ld_y,
+                                         float *state, int B, int D, int N, void *stream)
+{
+    const hyena_status_t st = check_packed(xp, ld_x, group, y, ld_y, B, 1, D);
+    if (st != HYENA_OK) return st;
+    return modal_decode_impl(packed_source(xp, ld_x, group), log_poles, residues, Dskip, y, ld_y, state, B, D, N,
+                             stream);
+}
+
+hyena_status_t hyena_short_decode(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
+                                  int64_t ld_x, const hyena_bf16_t *taps, const float *Dskip, hyena_bf16_t *y,
+                                  int64_t ld_y, float *hist, int B, int D, int K, void *stream)
+{
+    const hyena_status_t st = check_x(x1, x2, x3, ld_x, y, ld_y, B, 1, D);
+    if (st != HYENA_OK) return st;
+    return short_decode_impl(separate_source(x1, x2, x3, ld_x, D), taps, Dskip, y, ld_y, hist, B, D, K, stream);
+}
+
+hyena_status_t hyena_short_decode_packed(const hyena_bf16_t *xp, int64_t ld_x, int group, const hyena_bf16_t *taps,
+                                         const float *Dskip, hyena_bf16_t *y, int64_t ld_y, float *hist, int B,
+                                         int D, int K, void *stream)
+{
+    const hyena_status_t st = check_packed(xp, ld_x, group, y, ld_y, B, 1, D);
+    if (st != HYENA_OK) return st;
+    return short_decode_impl(packed_source(xp, ld_x, group), taps, Dskip, y, ld_y, hist, B, D, K, stream);
 }
 
 hyena_status_t hyena_modal_state_init(float *state, int B, int D, int N, void *stream)

@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(kDecodeThreads) modal_decode_kernel(const Deco
     if (idx >= static_cast<long long>(A.B) * A.D) return;
     const int b = static_cast<int>(idx / A.D);
     const int c = static_cast<int>(idx - static_cast<long long>(b) * A.D);
-    const size_t xi = static_cast<size_t>(b) * A.ld_x + c;
+    const size_t xi = static_cast<size_t>(b) * A.ld_x + x_col(c, A.group);
     const float v = __fmul_rn(bf16_bits_to_float(A.x1[xi]), bf16_bits_to_float(A.x2[xi]));
     const float x3 = bf16_bits_to_float(A.x3[xi]);
     float *st = A.state + (static_cast<size_t>(b) * A.D + c) * A.N;
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kDecodeThreads) fir_decode_kernel(const Decode
     const int b = static_cast<int>(idx / A.D);
     const int c = static_cast<int>(idx - static_cast<long long>(b) * A.D);
     const int K = A.K, H = K - 1;
-    const size_t xi = static_cast<size_t>(b) * A.ld_x + c;
+    const size_t xi = static_cast<size_t>(b) * A.ld_x + x_col(c, A.group);
     const float v = __fmul_rn(bf16_bits_to_float(A.x1[xi]), bf16_bits_to_float(A.x2[xi]));
     const float x3 = bf16_bits_to_float(A.x3[xi]);
     const uint16_t *tp = A.taps + static_cast<size_t>(c) * K;

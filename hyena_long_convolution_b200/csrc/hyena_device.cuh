@@ -96,6 +96,17 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// 4-D tiled TMA load (no multicast), as tma_load_3d with one more coordinate.
+__device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, uint64_t *bar,
+                                            int c0, int c1, int c2, int c3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // 2-D tiled TMA load (no multicast); c0 is the innermost coordinate and must
 // be 16-byte aligned in bytes.
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1)
@@ -135,6 +146,23 @@ __device__ __forceinline__ unsigned int ld_volatile_u32(const unsigned int *p)
 __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w)
 {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// Per-channel triples (x1_c, x2_c, x3_c adjacent): a channel pair (c, c+1)
+// occupies six bf16 values, x1_c x2_c x3_c x1_{c+1} x2_{c+1} x3_{c+1}, read as
+// three words w0 w1 w2 (lower address = low half).  Each helper returns the
+// pair (value of c, value of c+1) of one input; exact.
+__device__ __forceinline__ float2 tri_x1(uint32_t w0, uint32_t w1)
+{
+    return make_float2(__uint_as_float(w0 << 16), __uint_as_float(w1 & 0xffff0000u));
+}
+__device__ __forceinline__ float2 tri_x2(uint32_t w0, uint32_t w2)
+{
+    return make_float2(__uint_as_float(w0 & 0xffff0000u), __uint_as_float(w2 << 16));
+}
+__device__ __forceinline__ float2 tri_x3(uint32_t w1, uint32_t w2)
+{
+    return make_float2(__uint_as_float(w1 << 16), __uint_as_float(w2 & 0xffff0000u));
 }
 
 // Two fp32 values to two bf16 (round to nearest even), packed low = .x.

@@ -25,6 +25,20 @@ void record_message(const char *msg);
         }                                            \
     } while (0)
 
+// ---------------------------------------------------------------- inputs
+// Where x1, x2 and x3 live.  Channels come in groups of `group`; the row of
+// token t holds, for group g, the group's x1 values, then its x2 values, then
+// its x3 values, and x[k] points at element 0 of x_{k+1}.  Channel c of x_{k+1}
+// is therefore at column x_col(c, group) of x[k]:
+//   separate tensors  group = D, x[k] = the tensor (column c);
+//   packed, group G   x[k] = xp + k G (column 3G (c / G) + c % G);
+//   triples           group = 1, x[k] = xp + k (column 3c): the per-channel
+//                     interleave (x1_c, x2_c, x3_c adjacent).
+__host__ __device__ __forceinline__ long long x_col(int c, int group)
+{
+    return 3ll * group * (c / group) + c % group;
+}
+
 // ---------------------------------------------------------------- modal scan
 // A chain is the sequence of MCH channels of one batch row over time.  A unit
 // is MT consecutive tokens of a chain, swept by one warp (lane l owns the
@@ -54,6 +68,7 @@ ModalLayout modal_layout(int B, int D, int N);
 struct ModalArgs {
     const uint16_t *x3;
     long long ld_x;
+    int group;                  // channel group of the inputs (see x_col)
     uint16_t *y;
     long long ld_y;
     const float *state_in;
@@ -76,9 +91,11 @@ struct ModalSynthArgs {
 
 // Launches the coefficient-synthesis kernel and the scan kernel; returns the
 // number of launches enqueued or a negative value on a CUDA error.  The three
-// tensor maps cover x1, x2, x3 with [MCK x MCH] boxes.
+// 4-D tensor maps [B][L][groups][group] cover x1, x2, x3 with boxes of MCK rows
+// x MCH channels; with `triples` the first map alone covers the interleaved
+// rows (box MCK rows x 3 MCH elements) and the other two are unused.
 int launch_modal(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3,
-                 ModalArgs a, const ModalSynthArgs &s, int NP, cudaStream_t st);
+                 ModalArgs a, const ModalSynthArgs &s, int NP, bool triples, cudaStream_t st);
 
 // ---------------------------------------------------------------- short FIR
 constexpr int FCH = 64;   // channels per CTA
@@ -97,6 +114,7 @@ struct FirArgs {
     int B, L, D, K, HR;
     const uint16_t *x1, *x2;  // for the history kernel
     long long ld_x;
+    int group;                // channel group of the inputs (see x_col)
     float *hist_out;
 };
 
@@ -104,6 +122,7 @@ struct FirArgs {
 struct DecodeArgs {
     const uint16_t *x1, *x2, *x3;
     long long ld_x;
+    int group;                          // channel group of the inputs (see x_col)
     const float *log_poles, *residues;  // modal
     const uint16_t *taps;               // FIR
     const float *Dskip;
@@ -117,8 +136,11 @@ struct DecodeArgs {
 int launch_modal_decode(const DecodeArgs &a, cudaStream_t st);
 int launch_fir_decode(const DecodeArgs &a, cudaStream_t st);
 
+// Tile maps m1..m3 (FT rows) and halo maps h1, h2 (HR rows) over x1, x2, x3,
+// as for the modal scan; with `triples`, m1 and h1 alone cover the
+// interleaved rows.
 int launch_fir(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3,
                const CUtensorMap &h1, const CUtensorMap &h2, const FirArgs &a,
-               cudaStream_t st);
+               bool triples, cudaStream_t st);
 
 }  // namespace hyena

@@ -364,7 +364,11 @@ __device__ void control_warp(GroupSmem<NP, G> &sm, const ModalArgs &A, unsigned 
 // 0..7 carry x1/x2 rows of the unit for the A sweep, chunks 8..15 x1/x2/x3
 // rows for the C sweep.  Chunk q of warp w goes to buffer q % kRing once the
 // warp has released the chunk that used the buffer before.
-template <int NP, int G>
+// Separate or grouped inputs: one box of MCK rows x MCH channels per input
+// (x1, x2 for the A sweep, x1, x2, x3 for the C sweep) at 4-D coordinates
+// (column in group, group, token, batch row).  Triples: one box of MCK rows x
+// 3 MCH interleaved values holds all three inputs, for either sweep.
+template <int NP, int G, bool kTri>
 __device__ void producer_warp(GroupSmem<NP, G> &sm, const CUtensorMap *tm1, const CUtensorMap *tm2,
                               const CUtensorMap *tm3, const ModalArgs &A)
 {
@@ -372,6 +376,7 @@ __device__ void producer_warp(GroupSmem<NP, G> &sm, const CUtensorMap *tm1, cons
     const int lane = threadIdx.x & 31;
     int cur_k = -1;
     GroupPos q{};
+    int cx = 0, cg = 0;  // box coordinates of the group's channel block
     for (int qn = 0;; ++qn) {
         const int k = qn / kChunksPerGroup;
         const int c = qn % kChunksPerGroup;
@@ -380,6 +385,9 @@ __device__ void producer_warp(GroupSmem<NP, G> &sm, const CUtensorMap *tm1, cons
             const int gi = sm.gid[k & 1];
             if (gi < 0) break;
             q = group_pos(static_cast<unsigned int>(gi), A);
+            const int ch = q.cb * MCH;
+            cx = kTri ? 3 * ch : ch % A.group;
+            cg = kTri ? 0 : ch / A.group;
             cur_k = k;
         }
         const int b = qn % kRing;
@@ -390,20 +398,26 @@ __device__ void producer_warp(GroupSmem<NP, G> &sm, const CUtensorMap *tm1, cons
                 const int row = (static_cast<int>(q.s) * G + w) * MT + row_in_unit;
                 uint64_t *bar = &sm.full[w][b];
                 fence_proxy_async_smem();
-                if (c < kChunksPerSweep) {
-                    mbar_arrive_expect_tx(bar, 2 * kChunkBytes);
-                } else {
+                if constexpr (kTri) {
                     mbar_arrive_expect_tx(bar, 3 * kChunkBytes);
-                    tma_load_3d(sm.ring[w][b][2], tm3, bar, q.cb * MCH, row, q.b);
+                    tma_load_4d(sm.ring[w][b][0], tm1, bar, cx, 0, row, q.b);
+                } else {
+                    if (c < kChunksPerSweep) {
+                        mbar_arrive_expect_tx(bar, 2 * kChunkBytes);
+                    } else {
+                        mbar_arrive_expect_tx(bar, 3 * kChunkBytes);
+                        tma_load_4d(sm.ring[w][b][2], tm3, bar, cx, cg, row, q.b);
+                    }
+                    tma_load_4d(sm.ring[w][b][0], tm1, bar, cx, cg, row, q.b);
+                    tma_load_4d(sm.ring[w][b][1], tm2, bar, cx, cg, row, q.b);
                 }
-                tma_load_3d(sm.ring[w][b][0], tm1, bar, q.cb * MCH, row, q.b);
-                tma_load_3d(sm.ring[w][b][1], tm2, bar, q.cb * MCH, row, q.b);
             }
         }
     }
 }
 
 // ------------------------------------------------------------------ compute warps
+// Separate buffers: lane l reads word l of each 32-word row of x1, x2 (x3).
 template <int NP>
 __device__ __forceinline__ void sweep_a_chunk(float2 (&s)[NP], const float2 (&p)[NP], const uint32_t *r1,
                                               const uint32_t *r2)
@@ -416,17 +430,28 @@ __device__ __forceinline__ void sweep_a_chunk(float2 (&s)[NP], const float2 (&p)
     }
 }
 
+// Triples: rows of 96 words, the lane's three words at 3 l (x1/x2/x3 of its
+// channel pair interleaved).
+template <int NP>
+__device__ __forceinline__ void sweep_a_chunk_tri(float2 (&s)[NP], const float2 (&p)[NP], const uint32_t *rw)
+{
+#pragma unroll 4
+    for (int i = 0; i < MCK; ++i) {
+        const uint32_t w0 = rw[i * 96], w1 = rw[i * 96 + 1], w2 = rw[i * 96 + 2];
+        const float2 v = __fmul2_rn(tri_x1(w0, w1), tri_x2(w0, w2));
+#pragma unroll
+        for (int n = 0; n < NP; ++n) s[n] = __ffma2_rn(p[n], s[n], v);
+    }
+}
+
 // One token of the C sweep for this lane's channel pair: advance the N states,
 // form conv = sum_n R_n s_n with two independent accumulation chains (all
 // state updates first, so the chains find their inputs ready), apply the
 // gates and store y.
 template <int NP>
 __device__ __forceinline__ void sweep_c_token(float2 (&s)[NP], const float2 (&p)[NP], const float2 (&R)[NP],
-                                              float2 dsk, uint32_t w1, uint32_t w2, uint32_t w3,
-                                              uint32_t *yp, bool store)
+                                              float2 dsk, float2 v, float2 x3, uint32_t *yp, bool store)
 {
-    const float2 v = __fmul2_rn(bf16x2_to_float2(w1), bf16x2_to_float2(w2));
-    const float2 x3 = bf16x2_to_float2(w3);
 #pragma unroll
     for (int n = 0; n < NP; ++n) s[n] = __ffma2_rn(p[n], s[n], v);
     float2 a0 = __fmul2_rn(R[0], s[0]);
@@ -441,7 +466,23 @@ __device__ __forceinline__ void sweep_c_token(float2 (&s)[NP], const float2 (&p)
     st_pred_u32(yp, float2_to_bf16x2(yv), store);
 }
 
-template <int NP, int G>
+// v and x3 of row r of a chunk for this lane's channel pair.
+template <bool kTri>
+__device__ __forceinline__ void chunk_row(const uint32_t (&chunk)[3][kChunkWords], int lane, int r, float2 &v,
+                                          float2 &x3)
+{
+    if constexpr (kTri) {
+        const uint32_t *rw = &chunk[0][0] + r * 96 + 3 * lane;
+        const uint32_t w0 = rw[0], w1 = rw[1], w2 = rw[2];
+        v = __fmul2_rn(tri_x1(w0, w1), tri_x2(w0, w2));
+        x3 = tri_x3(w1, w2);
+    } else {
+        v = __fmul2_rn(bf16x2_to_float2(chunk[0][r * 32 + lane]), bf16x2_to_float2(chunk[1][r * 32 + lane]));
+        x3 = bf16x2_to_float2(chunk[2][r * 32 + lane]);
+    }
+}
+
+template <int NP, int G, bool kTri>
 __device__ void compute_warp(GroupSmem<NP, G> &sm, const ModalArgs &A)
 {
     constexpr int kRing = GroupTraits<G>::kRing;
@@ -469,7 +510,10 @@ __device__ void compute_warp(GroupSmem<NP, G> &sm, const ModalArgs &A)
         for (int i = 0; i < kChunksPerSweep; ++i, ++used) {
             const int b = used % kRing;
             (void)mbar_wait_tiles(&sm.full[w][b], (used / kRing) & 1, A.hdr);
-            sweep_a_chunk<NP>(s, p, sm.ring[w][b][0] + lane, sm.ring[w][b][1] + lane);
+            if constexpr (kTri)
+                sweep_a_chunk_tri<NP>(s, p, &sm.ring[w][b][0][0] + 3 * lane);
+            else
+                sweep_a_chunk<NP>(s, p, sm.ring[w][b][0] + lane, sm.ring[w][b][1] + lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[w][b]);
         }
@@ -503,18 +547,21 @@ __device__ void compute_warp(GroupSmem<NP, G> &sm, const ModalArgs &A)
         for (int i = 0; i < kChunksPerSweep; ++i, ++used) {
             const int b = used % kRing;
             (void)mbar_wait_tiles(&sm.full[w][b], (used / kRing) & 1, A.hdr);
-            const uint32_t *r1 = sm.ring[w][b][0] + lane;
-            const uint32_t *r2 = sm.ring[w][b][1] + lane;
-            const uint32_t *r3 = sm.ring[w][b][2] + lane;
             const int base = i * MCK;
             uint32_t *yc = yrow + static_cast<size_t>(base) * ystride;
             if (base + MCK <= nvalid) {
 #pragma unroll
-                for (int r = 0; r < MCK; ++r)
-                    sweep_c_token<NP>(s, p, R, dsk, r1[r * 32], r2[r * 32], r3[r * 32], yc + r * ystride, ch_ok);
+                for (int r = 0; r < MCK; ++r) {
+                    float2 v, x3;
+                    chunk_row<kTri>(sm.ring[w][b], lane, r, v, x3);
+                    sweep_c_token<NP>(s, p, R, dsk, v, x3, yc + r * ystride, ch_ok);
+                }
             } else {
-                for (int r = 0; r < MCK && base + r < nvalid; ++r)
-                    sweep_c_token<NP>(s, p, R, dsk, r1[r * 32], r2[r * 32], r3[r * 32], yc + r * ystride, ch_ok);
+                for (int r = 0; r < MCK && base + r < nvalid; ++r) {
+                    float2 v, x3;
+                    chunk_row<kTri>(sm.ring[w][b], lane, r, v, x3);
+                    sweep_c_token<NP>(s, p, R, dsk, v, x3, yc + r * ystride, ch_ok);
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[w][b]);
@@ -533,7 +580,7 @@ __device__ void compute_warp(GroupSmem<NP, G> &sm, const ModalArgs &A)
     }
 }
 
-template <int NP, int G>
+template <int NP, int G, bool kTri>
 __global__ void __launch_bounds__(GroupTraits<G>::kThreads, GroupTraits<G>::kCtasPerSm)
     modal_scan_kernel(const __grid_constant__ CUtensorMap tm1, const __grid_constant__ CUtensorMap tm2,
                       const __grid_constant__ CUtensorMap tm3, const ModalArgs A)
@@ -565,9 +612,9 @@ __global__ void __launch_bounds__(GroupTraits<G>::kThreads, GroupTraits<G>::kCta
     if (warp == G)
         control_warp<NP, G>(sm, A, epoch);
     else if (warp == G + 1)
-        producer_warp<NP, G>(sm, &tm1, &tm2, &tm3, A);
+        producer_warp<NP, G, kTri>(sm, &tm1, &tm2, &tm3, A);
     else
-        compute_warp<NP, G>(sm, A);
+        compute_warp<NP, G, kTri>(sm, A);
 
     // Every chunk the producer issued belongs to a group the compute warps
     // consumed in full, so no TMA is in flight here.
@@ -604,7 +651,7 @@ __global__ void modal_synth_kernel(const ModalSynthArgs S)
     if (n == 0) S.coef[2 * NP * row + c] = (c < S.D && S.Dskip != nullptr) ? S.Dskip[c] : 0.f;
 }
 
-template <int NP, int G>
+template <int NP, int G, bool kTri>
 int launch_scan(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3, ModalArgs a,
                 cudaStream_t st)
 {
@@ -615,10 +662,12 @@ int launch_scan(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap 
     const int smem = static_cast<int>(sizeof(GroupSmem<NP, G>));
     const int threads = GroupTraits<G>::kThreads;
     if (configured_device != dev) {
-        HYENA_TRY(cudaFuncSetAttribute(modal_scan_kernel<NP, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+        HYENA_TRY(cudaFuncSetAttribute(modal_scan_kernel<NP, G, kTri>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       smem),
                   "modal scan: set max dynamic shared memory");
         HYENA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "multiprocessor count");
-        HYENA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, modal_scan_kernel<NP, G>, threads, smem),
+        HYENA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, modal_scan_kernel<NP, G, kTri>, threads,
+                                                                smem),
                   "modal scan: occupancy");
         if (per_sm < 1) per_sm = 1;
         configured_device = dev;
@@ -627,12 +676,12 @@ int launch_scan(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap 
     a.nGroups = groups_per_chain * static_cast<unsigned int>(a.B) * static_cast<unsigned int>(a.nCB);
     const unsigned int slots = static_cast<unsigned int>(sms * per_sm);
     const unsigned int grid = a.nGroups < slots ? a.nGroups : slots;
-    modal_scan_kernel<NP, G><<<grid, threads, smem, st>>>(m1, m2, m3, a);
+    modal_scan_kernel<NP, G, kTri><<<grid, threads, smem, st>>>(m1, m2, m3, a);
     HYENA_TRY(cudaGetLastError(), "modal scan launch");
     return 1;
 }
 
-template <int NP>
+template <int NP, bool kTri>
 int launch_modal_np(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3, const ModalArgs &a,
                     const ModalSynthArgs &s, cudaStream_t st)
 {
@@ -645,19 +694,28 @@ int launch_modal_np(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensor
     if (cudaGetDevice(&dev) == cudaSuccess) (void)cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long chains = static_cast<long long>(a.B) * a.nCB;
     const long long groups4 = chains * ((a.units + 3) / 4);
-    const int n = groups4 >= 4ll * sms ? launch_scan<NP, 4>(m1, m2, m3, a, st) : launch_scan<NP, 2>(m1, m2, m3, a, st);
+    const int n = groups4 >= 4ll * sms ? launch_scan<NP, 4, kTri>(m1, m2, m3, a, st)
+                                       : launch_scan<NP, 2, kTri>(m1, m2, m3, a, st);
     return n < 0 ? n : n + 1;
 }
 
 }  // namespace
 
 int launch_modal(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3, ModalArgs a,
-                 const ModalSynthArgs &s, int NP, cudaStream_t st)
+                 const ModalSynthArgs &s, int NP, bool triples, cudaStream_t st)
 {
+    if (triples) {
+        switch (NP) {
+            case 4: return launch_modal_np<4, true>(m1, m2, m3, a, s, st);
+            case 8: return launch_modal_np<8, true>(m1, m2, m3, a, s, st);
+            case 16: return launch_modal_np<16, true>(m1, m2, m3, a, s, st);
+            default: return -1;
+        }
+    }
     switch (NP) {
-        case 4: return launch_modal_np<4>(m1, m2, m3, a, s, st);
-        case 8: return launch_modal_np<8>(m1, m2, m3, a, s, st);
-        case 16: return launch_modal_np<16>(m1, m2, m3, a, s, st);
+        case 4: return launch_modal_np<4, false>(m1, m2, m3, a, s, st);
+        case 8: return launch_modal_np<8, false>(m1, m2, m3, a, s, st);
+        case 16: return launch_modal_np<16, false>(m1, m2, m3, a, s, st);
         default: return -1;
     }
 }

@@ -214,6 +214,57 @@ hyena_status_t hyena_short_decode(const hyena_bf16_t *x1, const hyena_bf16_t *x2
                                   float *hist, int B, int D, int K, void *stream);
 
 /*
+ * Packed projection inputs.  The Hyena input projection writes one
+ * [B, L, 3D] output per block (evo2_flash README, hook table row
+ * "blocks.N.projections", the in_proj output of width 3H), and its Hyena
+ * channels are interleaved per triple (same README, §Limitations).  The
+ * *_packed entry points read x1, x2, x3 straight from such a buffer:
+ *
+ * xp     [B, L, ld_x] bf16, device, 16-byte aligned; ld_x >= 3D, ld_x % 8 == 0.
+ *        For decode, L = 1: row b at b * ld_x.
+ * group  channels per group.  Row (b, t) holds, for each group g of `group`
+ *        channels, the group's x1 values, then its x2 values, then its x3
+ *        values:
+ *          x_k[b, t, c] = xp[(b*L + t)*ld_x + 3*group*(c / group)
+ *                            + (k-1)*group + c % group],   k = 1, 2, 3.
+ *        group = 1 is the per-channel triple interleave (x1_c, x2_c, x3_c
+ *        adjacent); group = D is three [x1 | x2 | x3] blocks (the same as
+ *        passing the three views to the plain entry points).
+ *        Supported: group = 1, group = D, or group a multiple of 8 that
+ *        divides D and either divides 64 or is a multiple of 64.  group < 1
+ *        or D % group != 0 gives HYENA_ERR_INVALID_ARG, any other group
+ *        HYENA_ERR_UNSUPPORTED.
+ * Every other argument, the result (bit for bit) and the error behaviour are
+ * those of the plain entry point with the same name minus "_packed"; y must
+ * not overlap xp.
+ */
+hyena_status_t hyena_modal_long_conv_packed(const hyena_bf16_t *xp, int64_t ld_x, int group,
+                                            const float *log_poles, const float *residues,
+                                            const float *Dskip,
+                                            hyena_bf16_t *y, int64_t ld_y,
+                                            const float *state_in, float *state_out,
+                                            int B, int L, int D, int N,
+                                            void *workspace, size_t workspace_bytes,
+                                            void *stream);
+
+hyena_status_t hyena_short_conv_packed(const hyena_bf16_t *xp, int64_t ld_x, int group,
+                                       const hyena_bf16_t *taps, const float *Dskip,
+                                       hyena_bf16_t *y, int64_t ld_y,
+                                       const float *hist_in, float *hist_out,
+                                       int B, int L, int D, int K, void *stream);
+
+hyena_status_t hyena_modal_decode_packed(const hyena_bf16_t *xp, int64_t ld_x, int group,
+                                         const float *log_poles, const float *residues,
+                                         const float *Dskip,
+                                         hyena_bf16_t *y, int64_t ld_y,
+                                         float *state, int B, int D, int N, void *stream);
+
+hyena_status_t hyena_short_decode_packed(const hyena_bf16_t *xp, int64_t ld_x, int group,
+                                         const hyena_bf16_t *taps, const float *Dskip,
+                                         hyena_bf16_t *y, int64_t ld_y,
+                                         float *hist, int B, int D, int K, void *stream);
+
+/*
  * Zero-fills a modal state [B, D, N] fp32 (the state before the first token
  * of a sequence): the start of chunked prefill.
  */

@@ -125,6 +125,44 @@ def test_short_decode_rejects_bad_arguments(kw, code):
     assert fdec(hy.lib(), **kw) == code
 
 
+def packed_calls(lib, xp=A, ld_x=192, group=1, y=A + 65536, ld_y=64, B=1, L=16, D=64):
+    """Status of each packed entry point for one projection-buffer description
+    (every other argument valid)."""
+    return {
+        "modal": lib.hyena_modal_long_conv_packed(xp, ld_x, group, A, A, None, y, ld_y, None, None,
+                                                  B, L, D, 8, None, 0, None),
+        "fir": lib.hyena_short_conv_packed(xp, ld_x, group, A, None, y, ld_y, None, None, B, L, D, 7, None),
+        "mdec": lib.hyena_modal_decode_packed(xp, ld_x, group, A, A, None, y, ld_y, A, B, D, 8, None),
+        "fdec": lib.hyena_short_decode_packed(xp, ld_x, group, A, None, y, ld_y, A, B, D, 7, None),
+    }
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(group=0), INVALID), (dict(group=-8), INVALID), (dict(group=7), INVALID),  # 64 % 7 != 0
+    (dict(D=48, ld_x=144, ld_y=48, group=12), UNSUP),   # not a multiple of 8
+    (dict(D=48, ld_x=144, ld_y=48, group=24), UNSUP),   # neither divides 64 nor is a multiple of 64
+    (dict(D=192, ld_x=576, ld_y=192, group=96), UNSUP),
+    (dict(ld_x=184), INVALID), (dict(xp=None), INVALID), (dict(y=None), INVALID), (dict(B=0), INVALID),
+    (dict(xp=A + 2), ALIGN), (dict(ld_x=196), ALIGN), (dict(D=60, ld_x=180, ld_y=64, group=1), ALIGN),
+])
+def test_packed_entry_points_reject_bad_arguments(kw, code):
+    res = packed_calls(hy.lib(), **kw)
+    assert set(res.values()) == {code}, res
+
+
+def test_packed_entry_points_check_their_own_arguments():
+    """A valid buffer description with an invalid filter argument fails the
+    same way as the plain entry point."""
+    lib = hy.lib()
+    assert lib.hyena_modal_long_conv_packed(A, 192, 1, A, A, None, A + 65536, 64, None, None,
+                                            1, 16, 64, 17, None, 0, None) == UNSUP
+    assert lib.hyena_modal_long_conv_packed(A, 192, 64, A, A, None, A + 65536, 64, None, None,
+                                            1, 16, 64, 8, None, 0, None) == WORKSPACE
+    assert lib.hyena_short_conv_packed(A, 192, 8, A, None, A + 65536, 64, None, None, 1, 16, 64, 129, None) == UNSUP
+    assert lib.hyena_modal_decode_packed(A, 192, 16, A, A, None, A + 65536, 64, None, 1, 64, 8, None) == INVALID
+    assert lib.hyena_short_decode_packed(A, 192, 32, A, None, A + 65536, 64, None, 1, 64, 7, None) == INVALID
+
+
 def test_other_entry_points_reject_bad_arguments():
     lib = hy.lib()
     assert lib.hyena_modal_state_init(None, 1, 64, 8, None) == INVALID

@@ -51,7 +51,7 @@ def check(inp, hist_in=None, **kw):
 
 
 @pytest.mark.parametrize("K", [1, 2, 7, 8, 9, 15, 64, 127, 128])
-@pytest.mark.parametrize("B,L,D", [(1, 300, 64), (2, 257, 136)])
+@pytest.mark.parametrize("B,L,D", [(1, 300, 64), (2, 257, 136), (1, 130, 48)])
 def test_shapes(K, B, L, D):
     inp = make_fir_inputs(B, L, D, K, seed=K * 7 + L, with_skip=True)
     H = np.random.default_rng(K).standard_normal((B, K - 1, D)).astype(np.float32).astype(np.float64)

@@ -78,7 +78,7 @@ def test_config0_with_state_and_direct_form():
 
 @pytest.mark.parametrize("B,L,D,N", [
     (1, 1, 64, 16), (1, 2, 8, 1), (2, 127, 72, 3), (1, 128, 64, 8), (2, 129, 136, 16),
-    (3, 1000, 200, 5), (1, 2048, 64, 16), (2, 4100, 520, 12), (1, 40000, 64, 4),
+    (3, 1000, 200, 5), (1, 2048, 64, 16), (2, 4100, 520, 12), (1, 40000, 64, 4), (2, 300, 24, 4),
 ])
 def test_shapes_ragged(B, L, D, N):
     inp = make_modal_inputs(B, L, D, N, seed=B * 1000 + L + D + N)

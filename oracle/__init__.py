@@ -53,8 +53,11 @@ def _load():
             lib.hyena_oracle_modal_recurrence.argtypes = [I, I, I, I, P, P, P, I64, P, P, P, P, P, P]
             lib.hyena_oracle_modal_direct.argtypes = [I, I, I, I, P, P, P, I64, P, P, P, P, P, P, P, I]
             lib.hyena_oracle_fir.argtypes = [I, I, I, I, P, P, P, I64, P, P, P, P, P]
+            lib.hyena_oracle_cmodal_recurrence.argtypes = [I, I, I, I, P, P, P, I64, P, P, P, P, P, P]
+            lib.hyena_oracle_cmodal_direct.argtypes = [I, I, I, I, P, P, P, I64, P, P, P, P, P, P, P, I]
             for f in (lib.hyena_oracle_modal_recurrence, lib.hyena_oracle_modal_direct,
-                      lib.hyena_oracle_fir):
+                      lib.hyena_oracle_fir, lib.hyena_oracle_cmodal_recurrence,
+                      lib.hyena_oracle_cmodal_direct):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -144,6 +147,52 @@ def modal_direct(x1, x2, x3, log_poles, residues, Dskip=None, state_in=None):
     return y, Sout
 
 
+def cmodal_recurrence(x1, x2, x3, poles, residues, Dskip=None, state_in=None):
+    """Complex-mode long conv by per-mode complex recurrences (fp64).
+
+    poles, residues: fp32 [D, N, 2] (real, imaginary); the filter is
+    h[k] = Re sum_n R_n p_n^k.  state_in: float [B, D, N, 2] or None.
+    Returns (y fp64 [B, L, D], state_out fp64 [B, D, N, 2]).
+    """
+    (x1, x2, x3), B, L, ld = _xs(x1, x2, x3)
+    p = _f32(poles)
+    D, N, two = p.shape
+    if two != 2:
+        raise ValueError("poles must be [D, N, 2]")
+    R = _f32(residues, (D, N, 2))
+    Ds = _f32(Dskip, (D,))
+    Sin = _f64(state_in, (B, D, N, 2))
+    y = np.empty((B, L, D), dtype=np.float64)
+    Sout = np.empty((B, D, N, 2), dtype=np.float64)
+    rc = _load().hyena_oracle_cmodal_recurrence(B, L, D, N, _ptr(x1), _ptr(x2), _ptr(x3), ld,
+                                                _ptr(p), _ptr(R), _ptr(Ds), _ptr(Sin),
+                                                _ptr(y), _ptr(Sout))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return y, Sout
+
+
+def cmodal_direct(x1, x2, x3, poles, residues, Dskip=None, state_in=None):
+    """Complex-mode long conv as a direct O(L^2) convolution with the filter
+    taken from the polar form of each mode (independent of the recurrence)."""
+    (x1, x2, x3), B, L, ld = _xs(x1, x2, x3)
+    p = _f32(poles)
+    D, N, _ = p.shape
+    R = _f32(residues, (D, N, 2))
+    Ds = _f32(Dskip, (D,))
+    Sin = _f64(state_in, (B, D, N, 2))
+    y = np.empty((B, L, D), dtype=np.float64)
+    Sout = np.empty((B, D, N, 2), dtype=np.float64)
+    slots = max(1, min(os.cpu_count() or 1, B * D))
+    scratch = np.empty(max(1, 2 * L * slots), dtype=np.float64)
+    rc = _load().hyena_oracle_cmodal_direct(B, L, D, N, _ptr(x1), _ptr(x2), _ptr(x3), ld,
+                                            _ptr(p), _ptr(R), _ptr(Ds), _ptr(Sin),
+                                            _ptr(y), _ptr(Sout), _ptr(scratch), slots)
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return y, Sout
+
+
 def fir(x1, x2, x3, taps, Dskip=None, hist_in=None):
     """Explicit causal FIR (hcs/hcm) in fp64.
 
@@ -200,3 +249,17 @@ def fir_chunked(x1, x2, x3, taps, Dskip=None, hist_in=None, chunks=1024):
         ys.append(y)
         t0 += n
     return np.concatenate(ys, axis=1), H
+
+
+def cmodal_chunked(x1, x2, x3, poles, residues, Dskip=None, state_in=None, chunks=1024):
+    """Complex modes fed chunk by chunk, carrying the fp64 complex state."""
+    L = np.asarray(x1).shape[1]
+    ys = []
+    S = state_in
+    t0 = 0
+    for n in _splits(L, chunks):
+        y, S = cmodal_recurrence(x1[:, t0:t0 + n], x2[:, t0:t0 + n], x3[:, t0:t0 + n],
+                                 poles, residues, Dskip, S)
+        ys.append(y)
+        t0 += n
+    return np.concatenate(ys, axis=1), S

@@ -40,6 +40,7 @@
  * the other: a direct O(L^2) convolution with the synthesised filter, and a
  * first-order recurrence per mode.
  */
+#include <complex.h>
 #include <math.h>
 #include <stdint.h>
 #include <stddef.h>
@@ -169,6 +170,155 @@ int hyena_oracle_modal_direct(int B, int L, int D, int N,
                                           : 0.0;
                     for (int s = 0; s < L; ++s) acc += exp((double)ac[n] * (L - 1 - s)) * v[s];
                     state_out[((size_t)b * D + c) * N + n] = acc;
+                }
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * Complex modes (Evo1-1.5-7B-8K model card, §Architecture: modal-form
+ * "poles" / "residues" kept in fp32, Hyena state size 8).  Each mode n of
+ * channel c has a complex pole p and a complex residue R, given as fp32
+ * (real, imaginary) pairs, layout [D][N][2]; the filter is the real part of
+ * the modal sum,
+ *     h[k] = Re sum_n R[c,n] p[c,n]^k,   k >= 0,
+ * so a conjugate pair (p, R), (conj p, conj R) is one mode with residue 2R.
+ * The state is the complex R-free mode sum after the last token, layout
+ * [B][D][N][2].
+ *
+ * Recurrence form, in complex arithmetic:
+ *     s_n[-1] = state_in[b,c,n]  (0 when state_in is NULL)
+ *     s_n[t]  = p s_n[t-1] + v[t]
+ *     conv[t] = Re sum_n R_n s_n[t]
+ */
+int hyena_oracle_cmodal_recurrence(int B, int L, int D, int N,
+                                   const uint16_t *x1, const uint16_t *x2,
+                                   const uint16_t *x3, int64_t ld_x,
+                                   const float *poles, const float *residues,
+                                   const float *Dskip, const double *state_in,
+                                   double *y, double *state_out)
+{
+    if (check_common(B, L, D, ld_x, x1, x2, x3, y) || N < 1 || N > 256 || !poles ||
+        !residues)
+        return ORACLE_BAD_ARG;
+    const long long BD = (long long)B * D;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long long bc = 0; bc < BD; ++bc) {
+        const int b = (int)(bc / D), c = (int)(bc % D);
+        double complex p[256], R[256], s[256];
+        for (int n = 0; n < N; ++n) {
+            const size_t k = ((size_t)c * N + n) * 2;
+            p[n] = (double)poles[k] + I * (double)poles[k + 1];
+            R[n] = (double)residues[k] + I * (double)residues[k + 1];
+            const size_t q = (((size_t)b * D + c) * N + n) * 2;
+            s[n] = state_in ? state_in[q] + I * state_in[q + 1] : 0.0;
+        }
+        const double dk = Dskip ? (double)Dskip[c] : 0.0;
+        for (int t = 0; t < L; ++t) {
+            const size_t ix = ((size_t)b * L + t) * (size_t)ld_x + c;
+            const double v = bf16_bits_to_double(x1[ix]) * bf16_bits_to_double(x2[ix]);
+            double complex acc = 0.0;
+            for (int n = 0; n < N; ++n) {
+                s[n] = p[n] * s[n] + v;
+                acc += R[n] * s[n];
+            }
+            y[((size_t)b * L + t) * D + c] = bf16_bits_to_double(x3[ix]) * creal(acc) + dk * v;
+        }
+        if (state_out)
+            for (int n = 0; n < N; ++n) {
+                const size_t q = (((size_t)b * D + c) * N + n) * 2;
+                state_out[q] = creal(s[n]);
+                state_out[q + 1] = cimag(s[n]);
+            }
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * Direct form of the complex modes, from the polar form of each term (no
+ * complex arithmetic): with p = rho e^{i theta}, R = m e^{i phi},
+ *     Re(R p^k) = m rho^k cos(k theta + phi),
+ *     h[k] = sum_n m_n rho_n^k cos(k theta_n + phi_n),
+ * applied as a plain causal convolution; a carried state S = sigma e^{i psi}
+ * adds Re(R p^(t+1) S) = m sigma rho^(t+1) cos((t+1) theta + phi + psi), and
+ *     state_out = p^L S + sum_{s<L} p^(L-1-s) v[s]
+ * (real and imaginary parts from rho^k (cos, sin)(k theta)).  O(L^2).
+ */
+int hyena_oracle_cmodal_direct(int B, int L, int D, int N,
+                               const uint16_t *x1, const uint16_t *x2,
+                               const uint16_t *x3, int64_t ld_x,
+                               const float *poles, const float *residues,
+                               const float *Dskip, const double *state_in,
+                               double *y, double *state_out,
+                               double *scratch /* 2*L doubles per thread slot */,
+                               int scratch_slots)
+{
+    if (check_common(B, L, D, ld_x, x1, x2, x3, y) || N < 1 || !poles || !residues ||
+        (L > 0 && (!scratch || scratch_slots < 1)))
+        return ORACLE_BAD_ARG;
+    const long long BD = (long long)B * D;
+#pragma omp parallel for schedule(static, 1) num_threads(scratch_slots)
+    for (int slot = 0; slot < scratch_slots; ++slot) {
+        double *h = scratch + (size_t)slot * 2 * (size_t)L;
+        double *v = h + L;
+        for (long long bc = slot; bc < BD; bc += scratch_slots) {
+            const int b = (int)(bc / D), c = (int)(bc % D);
+            const float *pc = poles + (size_t)c * N * 2;
+            const float *rc = residues + (size_t)c * N * 2;
+            for (int k = 0; k < L; ++k) {
+                double acc = 0.0;
+                for (int n = 0; n < N; ++n) {
+                    const double rho = hypot(pc[2 * n], pc[2 * n + 1]);
+                    const double theta = atan2(pc[2 * n + 1], pc[2 * n]);
+                    const double m = hypot(rc[2 * n], rc[2 * n + 1]);
+                    const double phi = atan2(rc[2 * n + 1], rc[2 * n]);
+                    acc += m * pow(rho, k) * cos(k * theta + phi);
+                }
+                h[k] = acc;
+            }
+            for (int t = 0; t < L; ++t) {
+                const size_t ix = ((size_t)b * L + t) * (size_t)ld_x + c;
+                v[t] = bf16_bits_to_double(x1[ix]) * bf16_bits_to_double(x2[ix]);
+            }
+            const double dk = Dskip ? (double)Dskip[c] : 0.0;
+            for (int t = 0; t < L; ++t) {
+                double conv = 0.0;
+                for (int s = 0; s <= t; ++s) conv += h[t - s] * v[s];
+                if (state_in)
+                    for (int n = 0; n < N; ++n) {
+                        const size_t q = (((size_t)b * D + c) * N + n) * 2;
+                        const double rho = hypot(pc[2 * n], pc[2 * n + 1]);
+                        const double theta = atan2(pc[2 * n + 1], pc[2 * n]);
+                        const double m = hypot(rc[2 * n], rc[2 * n + 1]);
+                        const double phi = atan2(rc[2 * n + 1], rc[2 * n]);
+                        const double sigma = hypot(state_in[q], state_in[q + 1]);
+                        const double psi = atan2(state_in[q + 1], state_in[q]);
+                        conv += m * sigma * pow(rho, t + 1) * cos((t + 1) * theta + phi + psi);
+                    }
+                const size_t ix = ((size_t)b * L + t) * (size_t)ld_x + c;
+                y[((size_t)b * L + t) * D + c] = bf16_bits_to_double(x3[ix]) * conv + dk * v[t];
+            }
+            if (state_out) {
+                for (int n = 0; n < N; ++n) {
+                    const size_t q = (((size_t)b * D + c) * N + n) * 2;
+                    const double rho = hypot(pc[2 * n], pc[2 * n + 1]);
+                    const double theta = atan2(pc[2 * n + 1], pc[2 * n]);
+                    double re = 0.0, im = 0.0;
+                    if (state_in) {
+                        const double sigma = hypot(state_in[q], state_in[q + 1]);
+                        const double psi = atan2(state_in[q + 1], state_in[q]);
+                        re = sigma * pow(rho, L) * cos(L * theta + psi);
+                        im = sigma * pow(rho, L) * sin(L * theta + psi);
+                    }
+                    for (int s = 0; s < L; ++s) {
+                        const int k = L - 1 - s;
+                        re += pow(rho, k) * cos(k * theta) * v[s];
+                        im += pow(rho, k) * sin(k * theta) * v[s];
+                    }
+                    state_out[q] = re;
+                    state_out[q + 1] = im;
                 }
             }
         }

@@ -9,6 +9,7 @@ from .inputs import (  # noqa: F401
     CONFIGS,
     bf16_bits_to_f32,
     f32_to_bf16_bits,
+    make_cmodal_inputs,
     make_fir_inputs,
     make_inputs_for_config,
     make_modal_inputs,

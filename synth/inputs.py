@@ -19,6 +19,11 @@ Recipe (every config):
     multiplied by its factor in fp32 before rounding to bf16.
   * FIR taps from ``default_rng([seed, 101])``: N(0, 1/K) fp32 [D, K] rounded
     to bf16; FIR skip (when requested) from the same generator, N(0, 1).
+  * complex modal parameters from ``default_rng([seed, 102])``, in this order:
+    pole moduli r = exp(-exp(U(ln 1e-3, 0))) [D, N] (the real log-pole draw,
+    exponentiated), pole angles U(0, pi) [D, N], residues (N(0, 1) + i N(0, 1))
+    / sqrt(2N) [D, N], skip N(0, 1) [D]; poles r (cos, sin) and residues are
+    stored as fp32 [D, N, 2] (real, imaginary).
 
 All integer bit patterns are numpy uint16 arrays so the oracle and the GPU read
 identical bits.
@@ -113,6 +118,26 @@ def make_modal_params(seed: int, D: int, N: int, wide_range: bool = False):
     if wide_range:
         scales = (10.0 ** g.uniform(-2.0, 2.0, size=(3, D))).astype(np.float32)
     return a, R, Dskip, scales
+
+
+def make_cmodal_params(seed: int, D: int, N: int):
+    g = np.random.default_rng([seed, 102])
+    r = np.exp(-np.exp(g.uniform(math.log(1e-3), 0.0, size=(D, N))))
+    theta = g.uniform(0.0, math.pi, size=(D, N))
+    Rre = g.standard_normal((D, N))
+    Rim = g.standard_normal((D, N))
+    Dskip = g.standard_normal(D).astype(np.float32)
+    poles = np.stack([r * np.cos(theta), r * np.sin(theta)], axis=-1).astype(np.float32)
+    residues = (np.stack([Rre, Rim], axis=-1) / math.sqrt(2 * N)).astype(np.float32)
+    return poles, residues, Dskip
+
+
+def make_cmodal_inputs(B: int, L: int, D: int, N: int, seed: int, threads: int | None = None) -> dict:
+    """x1, x2, x3 as for the real modal filter; N complex modes (poles and
+    residues fp32 [D, N, 2])."""
+    poles, residues, Dskip = make_cmodal_params(seed, D, N)
+    x1, x2, x3 = make_x(seed, B, L, D, None, threads)
+    return dict(x1=x1, x2=x2, x3=x3, poles=poles, residues=residues, Dskip=Dskip, B=B, L=L, D=D, N=N)
 
 
 def make_modal_inputs(B: int, L: int, D: int, N: int, seed: int,

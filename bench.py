@@ -58,6 +58,11 @@ WORKLOADS = {
                          desc="hcs explicit FIR K=7, B=2 L=8192 D=4096, inputs interleaved per channel triple"),
     "fir128_triples": dict(kind="fir", B=2, L=8192, D=4096, K=128, seed=1, group=1,
                            desc="hcm explicit FIR K=128, B=2 L=8192 D=4096, inputs interleaved per channel triple"),
+    # complex modes, h[t] = Re sum R p^t (the Evo 1 modal form; state size 8)
+    "cmodal8k": dict(kind="modal", cx=True, B=1, L=8192, D=4096, N=8, seed=9, chunk=None,
+                     desc="complex-mode modal long conv, B=1 L=8192 D=4096 N=8, single pass"),
+    "cmodal32k": dict(kind="modal", cx=True, B=1, L=32768, D=4096, N=8, seed=10, chunk=None,
+                      desc="complex-mode modal long conv, B=1 L=32768 D=4096 N=8, single pass"),
     # generation: one step = L one-token decode calls (state / window carried)
     "decode_modal": dict(kind="modal", decode=True, B=1, L=256, D=4096, N=16, seed=5, chunk=None,
                          desc="hcl decode, B=1 D=4096 N=16, 256 one-token steps"),
@@ -98,8 +103,11 @@ def algorithmic_bytes(wl):
 
 def flops_per_chtok(wl):
     """Algorithmic flops per channel-token: the recurrence form's 2N FMAs
-    (hcl) or K FMAs (explicit FIR), plus v = x1 x2, the gate and the skip."""
-    return 4 * wl["N"] + 4 if wl["kind"] == "modal" else 2 * wl["K"] + 4
+    (hcl; complex modes: 6N, four for p s + v and two for Re(R s)) or K FMAs
+    (explicit FIR), plus v = x1 x2, the gate and the skip."""
+    if wl["kind"] == "modal":
+        return (12 if wl.get("cx") else 4) * wl["N"] + 4
+    return 2 * wl["K"] + 4
 
 
 def measured_peaks():
@@ -240,13 +248,19 @@ def oracle_sample_rate(wl, target_s=10.0):
     Returns (channel-tokens/s, sample description, threads).
     """
     import oracle
-    from synth import make_fir_inputs, make_modal_inputs
+    from synth import make_cmodal_inputs, make_fir_inputs, make_modal_inputs
     threads = oracle_threads()
     os.environ.setdefault("OMP_NUM_THREADS", str(threads))
     L = wl["L"]
     B = wl["B"]
 
     def run(D):
+        if wl.get("cx"):
+            inp = make_cmodal_inputs(B, L, D, wl["N"], wl["seed"])
+            t = time.perf_counter()
+            oracle.cmodal_recurrence(inp["x1"], inp["x2"], inp["x3"], inp["poles"], inp["residues"],
+                                     inp["Dskip"])
+            return time.perf_counter() - t
         if wl["kind"] == "modal":
             inp = make_modal_inputs(B, L, D, wl["N"], wl["seed"], wl.get("wide", False))
             t = time.perf_counter()
@@ -285,12 +299,19 @@ def oracle_sample_rate(wl, target_s=10.0):
 
 def make_device_inputs(wl, device):
     import torch
-    from synth import make_fir_inputs, make_modal_inputs
+    from synth import make_cmodal_inputs, make_fir_inputs, make_modal_inputs
 
     def up(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
 
-    if wl["kind"] == "modal":
+    if wl.get("cx"):
+        inp = make_cmodal_inputs(wl["B"], wl["L"], wl["D"], wl["N"], wl["seed"])
+        host = dict(x1=inp["x1"], x2=inp["x2"], x3=inp["x3"], a=inp["poles"], R=inp["residues"], Ds=inp["Dskip"])
+        dev = dict(x1=up(inp["x1"]), x2=up(inp["x2"]), x3=up(inp["x3"]),
+                   a=torch.from_numpy(inp["poles"]).to(device),
+                   R=torch.from_numpy(inp["residues"]).to(device),
+                   Ds=torch.from_numpy(inp["Dskip"]).to(device))
+    elif wl["kind"] == "modal":
         inp = make_modal_inputs(wl["B"], wl["L"], wl["D"], wl["N"], wl["seed"], wl.get("wide", False))
         host = dict(x1=inp["x1"], x2=inp["x2"], x3=inp["x3"])
         dev = dict(x1=up(inp["x1"]), x2=up(inp["x2"]), x3=up(inp["x3"]),
@@ -327,8 +348,9 @@ class Step:
         self.y = torch.empty((B, L, D), dtype=torch.bfloat16, device=device)
         self.launches = 0
         if wl["kind"] == "modal":
-            self.ws = hy.ModalWorkspace(B, D, wl["N"], device=device)
-            self.S = torch.zeros((B, D, wl["N"]), device=device)
+            cx = bool(wl.get("cx"))
+            self.ws = hy.ModalWorkspace(B, D, (2 if cx else 1) * wl["N"], device=device)
+            self.S = torch.zeros((B, D, wl["N"], 2) if cx else (B, D, wl["N"]), device=device)
         elif wl.get("decode"):
             self.H = torch.zeros((B, wl["K"] - 1, D), device=device)
         self.graph = None
@@ -364,6 +386,11 @@ class Step:
                                     y=self.y[:, sl])
                 n += hy.last_launch_count()
             self.launches = n
+            return
+        if wl.get("cx"):
+            hy.modal_long_conv_complex(d["x1"], d["x2"], d["x3"], d["a"], d["R"], d["Ds"], y=self.y,
+                                       state_out=self.S, workspace=self.ws)
+            self.launches = hy.last_launch_count()
             return
         if wl.get("group"):
             if wl["kind"] == "modal":
@@ -433,8 +460,9 @@ def e2e_leg(wl, host, dev, device, steps, warmup):
     B, L, D = wl["B"], wl["L"], wl["D"]
     y = torch.empty((B, L, D), dtype=torch.bfloat16, device=device)
     if wl["kind"] == "modal":
-        ws = hy.ModalWorkspace(B, D, wl["N"], device=device)
-        S = torch.zeros((B, D, wl["N"]), device=device)
+        cx = bool(wl.get("cx"))
+        ws = hy.ModalWorkspace(B, D, (2 if cx else 1) * wl["N"], device=device)
+        S = torch.zeros((B, D, wl["N"], 2) if cx else (B, D, wl["N"]), device=device)
     elif wl.get("decode"):
         H = torch.zeros((B, wl["K"] - 1, D), device=device)
 
@@ -442,7 +470,9 @@ def e2e_leg(wl, host, dev, device, steps, warmup):
         for k in hx:
             dx[k].copy_(hx[k], non_blocking=True)
         bf = {k: dx[k].view(torch.bfloat16) for k in ("x1", "x2", "x3", "xp") if k in dx}
-        if wl.get("group"):
+        if wl.get("cx"):
+            hy.modal_long_conv_complex(bf["x1"], bf["x2"], bf["x3"], dx["a"], dx["R"], dx["Ds"], y=y, workspace=ws)
+        elif wl.get("group"):
             if wl["kind"] == "modal":
                 hy.modal_long_conv_packed(bf["xp"], wl["group"], dx["a"], dx["R"], dx["Ds"], y=y, workspace=ws)
             else:
@@ -556,7 +586,8 @@ def run_gpu(args, wl):
         "io_dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 inputs, pages' shapes)",
         "config": {"workload": wl["desc"], "B": wl["B"], "L": wl["L"], "D": wl["D"],
-                   **({"N": wl["N"]} if wl["kind"] == "modal" else {"K": wl["K"]}),
+                   **({"N": wl["N"], "modes": "complex" if wl.get("cx") else "real"} if wl["kind"] == "modal"
+                      else {"K": wl["K"]}),
                    "mode": "decode (one-token calls)" if wl.get("decode") else "prefill",
                    "input_layout": (f"packed projection, channel groups of {wl['group']}" if wl.get("group")
                                     else "three [B, L, D] tensors"),

@@ -26,8 +26,10 @@ __all__ = [
     "ModalWorkspace",
     "last_launch_count",
     "modal_decode",
+    "modal_decode_complex",
     "modal_decode_packed",
     "modal_long_conv",
+    "modal_long_conv_complex",
     "modal_long_conv_packed",
     "modal_state_init",
     "short_conv",
@@ -39,6 +41,7 @@ __all__ = [
 ]
 
 MAX_MODES = 16
+MAX_COMPLEX_MODES = 8
 MAX_TAPS = 128
 
 
@@ -367,4 +370,72 @@ def short_decode_packed(xp, group, taps, Dskip, hist, y=None, stream=None):
     rc = lib().hyena_short_decode_packed(_ptr(xp), ld, int(group), _ptr(taps), _ptr(Dskip), _ptr(y), ld_y,
                                          _ptr(hist) if K > 1 else None, B, D, K, _stream(stream))
     check("hyena_short_decode_packed", rc)
+    return y
+
+
+# ---------------------------------------------------------------- complex modes
+
+def _cpar(poles, residues):
+    """poles, residues fp32 [D, N, 2] (real, imaginary) -> (D, N)."""
+    if poles.dim() != 3 or poles.shape[2] != 2:
+        raise ValueError("poles must be a [D, N, 2] fp32 tensor")
+    D, N, _ = poles.shape
+    _f32(poles, (D, N, 2), "poles", False)
+    _f32(residues, (D, N, 2), "residues", False)
+    return D, N
+
+
+def modal_long_conv_complex(x1, x2, x3, poles, residues, Dskip=None, y=None, state_in=None,
+                            state_out=None, workspace: ModalWorkspace | None = None, stream=None):
+    """Long modal filter with complex modes, h[t] = Re sum_n R_n p_n^t, with
+    fused gates.  poles, residues: [D, N, 2] fp32 (real, imaginary);
+    state_in/state_out: [B, D, N, 2] fp32 or None.  The workspace is that of
+    2N real modes."""
+    torch = _torch()
+    s1, s2, s3 = _bld(x1, "x1"), _bld(x2, "x2"), _bld(x3, "x3")
+    _same_ld(s1, s2, s3)
+    B, L, D, ld = s1
+    if s2[:3] != (B, L, D) or s3[:3] != (B, L, D):
+        raise ValueError("x1, x2, x3 shapes differ")
+    Dp, N = _cpar(poles, residues)
+    if Dp != D:
+        raise ValueError("poles must be [D, N, 2]")
+    _f32(Dskip, (D,), "Dskip")
+    _f32(state_in, (B, D, N, 2), "state_in")
+    _f32(state_out, (B, D, N, 2), "state_out")
+    if y is None:
+        y = torch.empty((B, L, D), dtype=torch.bfloat16, device=x1.device)
+    yB, yL, yD, ld_y = _bld(y, "y")
+    if (yB, yL, yD) != (B, L, D):
+        raise ValueError("y shape differs from x")
+    if workspace is None:
+        workspace = ModalWorkspace(B, D, 2 * N, device=x1.device, stream=stream)
+    rc = lib().hyena_modal_long_conv_complex(_ptr(x1), _ptr(x2), _ptr(x3), ld, _ptr(poles), _ptr(residues),
+                                             _ptr(Dskip), _ptr(y), ld_y, _ptr(state_in), _ptr(state_out),
+                                             B, L, D, N, _ptr(workspace.buf), workspace.nbytes, _stream(stream))
+    check("hyena_modal_long_conv_complex", rc)
+    return y
+
+
+def modal_decode_complex(x1, x2, x3, poles, residues, Dskip, state, y=None, stream=None):
+    """One generated token through the complex-mode filter: advances
+    ``state`` ([B, D, N, 2] fp32, in place); equals ``modal_long_conv_complex``
+    on a one-token sequence bit for bit."""
+    torch = _torch()
+    (B, D, ld), b2, b3 = _bd(x1, "x1"), _bd(x2, "x2"), _bd(x3, "x3")
+    if b2 != (B, D, ld) or b3 != (B, D, ld):
+        raise ValueError("x1, x2, x3 must share shape and row stride")
+    Dp, N = _cpar(poles, residues)
+    if Dp != D:
+        raise ValueError("poles must be [D, N, 2]")
+    _f32(Dskip, (D,), "Dskip")
+    _f32(state, (B, D, N, 2), "state", False)
+    if y is None:
+        y = torch.empty_like(x1, memory_format=torch.contiguous_format)
+    yB, yD, ld_y = _bd(y, "y")
+    if (yB, yD) != (B, D):
+        raise ValueError("y shape differs from x")
+    rc = lib().hyena_modal_decode_complex(_ptr(x1), _ptr(x2), _ptr(x3), ld, _ptr(poles), _ptr(residues),
+                                          _ptr(Dskip), _ptr(y), ld_y, _ptr(state), B, D, N, _stream(stream))
+    check("hyena_modal_decode_complex", rc)
     return y

@@ -237,14 +237,17 @@ hyena_status_t short_conv_impl(const XSource &xs, const hyena_bf16_t *taps, cons
     return HYENA_OK;
 }
 
+// cx: complex modes; the N of the caller counts modes, the kernels count
+// slots (two per complex mode).
 hyena_status_t modal_long_conv_impl(const XSource &xs, const float *log_poles, const float *residues,
                                    const float *Dskip, hyena_bf16_t *y, int64_t ld_y, const float *state_in,
                                    float *state_out, int B, int L, int D, int N, void *workspace,
-                                   size_t workspace_bytes, void *stream)
+                                   size_t workspace_bytes, void *stream, bool cx = false)
 {
     hyena_status_t st = HYENA_OK;
     if (N < 1) return HYENA_ERR_INVALID_ARG;
-    if (N > HYENA_MAX_MODES) return HYENA_ERR_UNSUPPORTED;
+    if (N > (cx ? HYENA_MAX_COMPLEX_MODES : HYENA_MAX_MODES)) return HYENA_ERR_UNSUPPORTED;
+    if (cx) N *= 2;
     if (!log_poles || !residues) return HYENA_ERR_INVALID_ARG;
     if (!aligned16(log_poles) || !aligned16(residues) || (Dskip && !aligned16(Dskip)) ||
         (state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
@@ -299,7 +302,7 @@ hyena_status_t modal_long_conv_impl(const XSource &xs, const float *log_poles, c
         m2 = m3 = m1;
     else if (!encode_x_map(&m2, xs, 1, B, L, D, MCK) || !encode_x_map(&m3, xs, 2, B, L, D, MCK))
         return HYENA_ERR_CUDA;
-    const int n = launch_modal(m1, m2, m3, a, sy, lay.NP, xs.triples, s);
+    const int n = launch_modal(m1, m2, m3, a, sy, lay.NP, xs.triples, cx, s);
     if (n < 0) return HYENA_ERR_CUDA;
     g_last_launches = n;
     return HYENA_OK;
@@ -307,9 +310,11 @@ hyena_status_t modal_long_conv_impl(const XSource &xs, const float *log_poles, c
 
 hyena_status_t modal_decode_impl(const XSource &xs, const float *log_poles, const float *residues,
                                  const float *Dskip, hyena_bf16_t *y, int64_t ld_y, float *state, int B, int D, int N,
-                                 void *stream)
+                                 void *stream, bool cx = false)
 {
-    if (N < 1 || N > HYENA_MAX_MODES) return N < 1 ? HYENA_ERR_INVALID_ARG : HYENA_ERR_UNSUPPORTED;
+    const int nmax = cx ? HYENA_MAX_COMPLEX_MODES : HYENA_MAX_MODES;
+    if (N < 1 || N > nmax) return N < 1 ? HYENA_ERR_INVALID_ARG : HYENA_ERR_UNSUPPORTED;
+    if (cx) N *= 2;
     if (!log_poles || !residues || !state) return HYENA_ERR_INVALID_ARG;
     if (!aligned16(log_poles) || !aligned16(residues) || !aligned16(state) || (Dskip && !aligned16(Dskip)))
         return HYENA_ERR_ALIGNMENT;
@@ -328,7 +333,7 @@ hyena_status_t modal_decode_impl(const XSource &xs, const float *log_poles, cons
     a.B = B;
     a.D = D;
     a.N = N;
-    const int n = launch_modal_decode(a, static_cast<cudaStream_t>(stream));
+    const int n = launch_modal_decode(a, cx, static_cast<cudaStream_t>(stream));
     if (n < 0) return HYENA_ERR_CUDA;
     g_last_launches = n;
     return HYENA_OK;
@@ -461,6 +466,29 @@ hyena_status_t hyena_modal_decode_packed(const hyena_bf16_t *xp, int64_t ld_x, i
     if (st != HYENA_OK) return st;
     return modal_decode_impl(packed_source(xp, ld_x, group), log_poles, residues, Dskip, y, ld_y, state, B, D, N,
                              stream);
+}
+
+hyena_status_t hyena_modal_long_conv_complex(const hyena_bf16_t *x1, const hyena_bf16_t *x2,
+                                             const hyena_bf16_t *x3, int64_t ld_x, const float *poles,
+                                             const float *residues, const float *Dskip, hyena_bf16_t *y,
+                                             int64_t ld_y, const float *state_in, float *state_out, int B, int L,
+                                             int D, int N, void *workspace, size_t workspace_bytes, void *stream)
+{
+    const hyena_status_t st = check_x(x1, x2, x3, ld_x, y, ld_y, B, L, D);
+    if (st != HYENA_OK) return st;
+    return modal_long_conv_impl(separate_source(x1, x2, x3, ld_x, D), poles, residues, Dskip, y, ld_y, state_in,
+                                state_out, B, L, D, N, workspace, workspace_bytes, stream, true);
+}
+
+hyena_status_t hyena_modal_decode_complex(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
+                                          int64_t ld_x, const float *poles, const float *residues,
+                                          const float *Dskip, hyena_bf16_t *y, int64_t ld_y, float *state, int B,
+                                          int D, int N, void *stream)
+{
+    const hyena_status_t st = check_x(x1, x2, x3, ld_x, y, ld_y, B, 1, D);
+    if (st != HYENA_OK) return st;
+    return modal_decode_impl(separate_source(x1, x2, x3, ld_x, D), poles, residues, Dskip, y, ld_y, state, B, D, N,
+                             stream, true);
 }
 
 hyena_status_t hyena_short_decode(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,

@@ -53,7 +53,10 @@ __device__ __forceinline__ void load_row(float (&v)[NP], const float *p, int N)
     }
 }
 
-template <int NP>
+// kCx: complex modes, N counts slots (two per mode, as the prefill kernel's
+// coefficient table): the pole pair is used as given and the residue pair as
+// (Re R, -Im R); the state update is the prefill kernel's complex step.
+template <int NP, bool kCx>
 __global__ void __launch_bounds__(kDecodeThreads) modal_decode_kernel(const DecodeArgs A)
 {
     const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -82,8 +85,19 @@ __global__ void __launch_bounds__(kDecodeThreads) modal_decode_kernel(const Deco
 #pragma unroll
         for (int i = 0; i < NP; ++i) s[i] = i < A.N ? st[i] : 0.f;
     }
+    if constexpr (!kCx) {
 #pragma unroll
-    for (int n = 0; n < NP; ++n) s[n] = __fmaf_rn(n < A.N ? expf(a[n]) : 0.f, s[n], v);
+        for (int n = 0; n < NP; ++n) s[n] = __fmaf_rn(n < A.N ? expf(a[n]) : 0.f, s[n], v);
+    } else {
+        // a[] holds the poles (zero in padded slots); residue pairs (Re, -Im)
+#pragma unroll
+        for (int m = 0; m < NP; m += 2) {
+            r[m + 1] = -r[m + 1];
+            const float re = s[m], im = s[m + 1];
+            s[m] = __fmaf_rn(a[m], re, __fmaf_rn(-a[m + 1], im, v));
+            s[m + 1] = __fmaf_rn(a[m], im, __fmul_rn(a[m + 1], re));
+        }
+    }
     float a0 = __fmul_rn(r[0], s[0]);
     float a1 = __fmul_rn(r[1], s[1]);
 #pragma unroll
@@ -157,14 +171,17 @@ __global__ void __launch_bounds__(kDecodeThreads) fir_decode_kernel(const Decode
 
 }  // namespace
 
-int launch_modal_decode(const DecodeArgs &a, cudaStream_t st)
+int launch_modal_decode(const DecodeArgs &a, bool cx, cudaStream_t st)
 {
     const long long n = static_cast<long long>(a.B) * a.D;
     const unsigned int grid = static_cast<unsigned int>((n + kDecodeThreads - 1) / kDecodeThreads);
-    switch (modal_padded_modes(a.N)) {
-        case 4: modal_decode_kernel<4><<<grid, kDecodeThreads, 0, st>>>(a); break;
-        case 8: modal_decode_kernel<8><<<grid, kDecodeThreads, 0, st>>>(a); break;
-        default: modal_decode_kernel<16><<<grid, kDecodeThreads, 0, st>>>(a); break;
+    switch (modal_padded_modes(a.N) + (cx ? 1 : 0)) {
+        case 4: modal_decode_kernel<4, false><<<grid, kDecodeThreads, 0, st>>>(a); break;
+        case 8: modal_decode_kernel<8, false><<<grid, kDecodeThreads, 0, st>>>(a); break;
+        case 16: modal_decode_kernel<16, false><<<grid, kDecodeThreads, 0, st>>>(a); break;
+        case 5: modal_decode_kernel<4, true><<<grid, kDecodeThreads, 0, st>>>(a); break;
+        case 9: modal_decode_kernel<8, true><<<grid, kDecodeThreads, 0, st>>>(a); break;
+        default: modal_decode_kernel<16, true><<<grid, kDecodeThreads, 0, st>>>(a); break;
     }
     HYENA_TRY(cudaGetLastError(), "modal decode launch");
     return 1;

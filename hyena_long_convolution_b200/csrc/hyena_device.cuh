@@ -172,6 +172,47 @@ __device__ __forceinline__ uint32_t float2_to_bf16x2(float2 f)
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// ---------------------------------------------------------------- modal modes
+// A lane's state of NP mode slots for its channel pair.  Real modes: slot n is
+// mode n.  Complex modes (pole p = pr + i pi): slots 2m and 2m+1 hold the real
+// and imaginary parts of mode m, of the state as of the pole.
+
+// One token, s <- p s + v with real v (packed f32x2 over the channel pair).
+template <int NP, bool kCx>
+__device__ __forceinline__ void modes_step(float2 (&s)[NP], const float2 (&p)[NP], float2 v)
+{
+    if constexpr (!kCx) {
+#pragma unroll
+        for (int n = 0; n < NP; ++n) s[n] = __ffma2_rn(p[n], s[n], v);
+    } else {
+#pragma unroll
+        for (int m = 0; m < NP; m += 2) {
+            const float2 re = s[m], im = s[m + 1];
+            const float2 npi = make_float2(-p[m + 1].x, -p[m + 1].y);
+            s[m] = __ffma2_rn(p[m], re, __ffma2_rn(npi, im, v));
+            s[m + 1] = __ffma2_rn(p[m], im, __fmul2_rn(p[m + 1], re));
+        }
+    }
+}
+
+// One carry step, C <- P C + A with a full state A (P = p^MT).
+template <int NP, bool kCx>
+__device__ __forceinline__ void modes_carry(float2 (&C)[NP], const float2 (&P)[NP], const float2 (&A)[NP])
+{
+    if constexpr (!kCx) {
+#pragma unroll
+        for (int n = 0; n < NP; ++n) C[n] = __ffma2_rn(P[n], C[n], A[n]);
+    } else {
+#pragma unroll
+        for (int m = 0; m < NP; m += 2) {
+            const float2 re = C[m], im = C[m + 1];
+            const float2 npi = make_float2(-P[m + 1].x, -P[m + 1].y);
+            C[m] = __ffma2_rn(P[m], re, __ffma2_rn(npi, im, A[m]));
+            C[m + 1] = __ffma2_rn(P[m], im, __ffma2_rn(P[m + 1], re, A[m + 1]));
+        }
+    }
+}
+
 __device__ __forceinline__ float2 ldg_f2(const float *p)
 {
     return __ldg(reinterpret_cast<const float2 *>(p));

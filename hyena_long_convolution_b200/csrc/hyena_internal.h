@@ -83,6 +83,9 @@ struct ModalArgs {
     unsigned int *hdr;          // [0] ticket, [1] finished CTAs, [2] error bits, [3] epoch
 };
 
+// Real modes: log_poles [D][N], residues [D][N].  Complex modes: log_poles
+// holds the poles and residues the residues as [D][N/2][2] (N counts slots,
+// two per complex mode).
 struct ModalSynthArgs {
     const float *log_poles, *residues, *Dskip;
     int D, N, Dp;
@@ -94,8 +97,10 @@ struct ModalSynthArgs {
 // 4-D tensor maps [B][L][groups][group] cover x1, x2, x3 with boxes of MCK rows
 // x MCH channels; with `triples` the first map alone covers the interleaved
 // rows (box MCK rows x 3 MCH elements) and the other two are unused.
+// With `cx` the N of the arguments counts mode slots, two per complex mode
+// (state [B][D][N/2][2] = [B][D][N]).
 int launch_modal(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3,
-                 ModalArgs a, const ModalSynthArgs &s, int NP, bool triples, cudaStream_t st);
+                 ModalArgs a, const ModalSynthArgs &s, int NP, bool triples, bool cx, cudaStream_t st);
 
 // ---------------------------------------------------------------- short FIR
 constexpr int FCH = 64;   // channels per CTA
@@ -133,7 +138,7 @@ struct DecodeArgs {
     int B, D, N, K;
 };
 
-int launch_modal_decode(const DecodeArgs &a, cudaStream_t st);
+int launch_modal_decode(const DecodeArgs &a, bool cx, cudaStream_t st);
 int launch_fir_decode(const DecodeArgs &a, cudaStream_t st);
 
 // Tile maps m1..m3 (FT rows) and halo maps h1, h2 (HR rows) over x1, x2, x3,

@@ -189,7 +189,7 @@ __device__ __forceinline__ void announce_group(GroupSmem<NP, G> &sm, const Modal
     }
 }
 
-template <int NP, int G>
+template <int NP, int G, bool kCx>
 __device__ void control_warp(GroupSmem<NP, G> &sm, const ModalArgs &A, unsigned int epoch)
 {
     const int lane = threadIdx.x & 31;
@@ -311,10 +311,8 @@ __device__ void control_warp(GroupSmem<NP, G> &sm, const ModalArgs &A, unsigned 
                         a[n] = __ldcg(reinterpret_cast<const float2 *>(src + (static_cast<size_t>(w) * NP + n) * MCH));
                         b2[n] = __ldcg(reinterpret_cast<const float2 *>(src + (static_cast<size_t>(w + 1) * NP + n) * MCH));
                     }
-#pragma unroll
-                    for (int n = 0; n < NP; ++n) C[n] = __ffma2_rn(pT[n], C[n], a[n]);
-#pragma unroll
-                    for (int n = 0; n < NP; ++n) C[n] = __ffma2_rn(pT[n], C[n], b2[n]);
+                    modes_carry<NP, kCx>(C, pT, a);
+                    modes_carry<NP, kCx>(C, pT, b2);
                 }
             }
         }
@@ -323,12 +321,13 @@ __device__ void control_warp(GroupSmem<NP, G> &sm, const ModalArgs &A, unsigned 
         {
             const bool whole_last = (A.L % MT) == 0;
             for (int w = 0; w < nvalid_units; ++w) {
+                float2 a[NP];
 #pragma unroll
                 for (int n = 0; n < NP; ++n) {
-                    const float2 a = sm.ac[w][n * 32 + lane];
+                    a[n] = sm.ac[w][n * 32 + lane];
                     sm.ac[w][n * 32 + lane] = C[n];
-                    C[n] = __ffma2_rn(pT[n], C[n], a);
                 }
+                modes_carry<NP, kCx>(C, pT, a);
                 // A sequence ending on a unit boundary takes its final state
                 // from the canonical chain (the expression a later chunk
                 // starts from).
@@ -418,42 +417,40 @@ __device__ void producer_warp(GroupSmem<NP, G> &sm, const CUtensorMap *tm1, cons
 
 // ------------------------------------------------------------------ compute warps
 // Separate buffers: lane l reads word l of each 32-word row of x1, x2 (x3).
-template <int NP>
+template <int NP, bool kCx>
 __device__ __forceinline__ void sweep_a_chunk(float2 (&s)[NP], const float2 (&p)[NP], const uint32_t *r1,
                                               const uint32_t *r2)
 {
 #pragma unroll 4
     for (int i = 0; i < MCK; ++i) {
         const float2 v = __fmul2_rn(bf16x2_to_float2(r1[i * 32]), bf16x2_to_float2(r2[i * 32]));
-#pragma unroll
-        for (int n = 0; n < NP; ++n) s[n] = __ffma2_rn(p[n], s[n], v);
+        modes_step<NP, kCx>(s, p, v);
     }
 }
 
 // Triples: rows of 96 words, the lane's three words at 3 l (x1/x2/x3 of its
 // channel pair interleaved).
-template <int NP>
+template <int NP, bool kCx>
 __device__ __forceinline__ void sweep_a_chunk_tri(float2 (&s)[NP], const float2 (&p)[NP], const uint32_t *rw)
 {
 #pragma unroll 4
     for (int i = 0; i < MCK; ++i) {
         const uint32_t w0 = rw[i * 96], w1 = rw[i * 96 + 1], w2 = rw[i * 96 + 2];
         const float2 v = __fmul2_rn(tri_x1(w0, w1), tri_x2(w0, w2));
-#pragma unroll
-        for (int n = 0; n < NP; ++n) s[n] = __ffma2_rn(p[n], s[n], v);
+        modes_step<NP, kCx>(s, p, v);
     }
 }
 
 // One token of the C sweep for this lane's channel pair: advance the N states,
 // form conv = sum_n R_n s_n with two independent accumulation chains (all
 // state updates first, so the chains find their inputs ready), apply the
-// gates and store y.
-template <int NP>
+// gates and store y.  Complex modes: the table holds (Re R, -Im R) in the
+// slot pair, so the same sum is Re sum_m R_m s_m.
+template <int NP, bool kCx>
 __device__ __forceinline__ void sweep_c_token(float2 (&s)[NP], const float2 (&p)[NP], const float2 (&R)[NP],
                                               float2 dsk, float2 v, float2 x3, uint32_t *yp, bool store)
 {
-#pragma unroll
-    for (int n = 0; n < NP; ++n) s[n] = __ffma2_rn(p[n], s[n], v);
+    modes_step<NP, kCx>(s, p, v);
     float2 a0 = __fmul2_rn(R[0], s[0]);
     float2 a1 = __fmul2_rn(R[1], s[1]);
 #pragma unroll
@@ -482,7 +479,7 @@ __device__ __forceinline__ void chunk_row(const uint32_t (&chunk)[3][kChunkWords
     }
 }
 
-template <int NP, int G, bool kTri>
+template <int NP, int G, bool kTri, bool kCx>
 __device__ void compute_warp(GroupSmem<NP, G> &sm, const ModalArgs &A)
 {
     constexpr int kRing = GroupTraits<G>::kRing;
@@ -511,9 +508,9 @@ __device__ void compute_warp(GroupSmem<NP, G> &sm, const ModalArgs &A)
             const int b = used % kRing;
             (void)mbar_wait_tiles(&sm.full[w][b], (used / kRing) & 1, A.hdr);
             if constexpr (kTri)
-                sweep_a_chunk_tri<NP>(s, p, &sm.ring[w][b][0][0] + 3 * lane);
+                sweep_a_chunk_tri<NP, kCx>(s, p, &sm.ring[w][b][0][0] + 3 * lane);
             else
-                sweep_a_chunk<NP>(s, p, sm.ring[w][b][0] + lane, sm.ring[w][b][1] + lane);
+                sweep_a_chunk<NP, kCx>(s, p, sm.ring[w][b][0] + lane, sm.ring[w][b][1] + lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[w][b]);
         }
@@ -554,13 +551,13 @@ __device__ void compute_warp(GroupSmem<NP, G> &sm, const ModalArgs &A)
                 for (int r = 0; r < MCK; ++r) {
                     float2 v, x3;
                     chunk_row<kTri>(sm.ring[w][b], lane, r, v, x3);
-                    sweep_c_token<NP>(s, p, R, dsk, v, x3, yc + r * ystride, ch_ok);
+                    sweep_c_token<NP, kCx>(s, p, R, dsk, v, x3, yc + r * ystride, ch_ok);
                 }
             } else {
                 for (int r = 0; r < MCK && base + r < nvalid; ++r) {
                     float2 v, x3;
                     chunk_row<kTri>(sm.ring[w][b], lane, r, v, x3);
-                    sweep_c_token<NP>(s, p, R, dsk, v, x3, yc + r * ystride, ch_ok);
+                    sweep_c_token<NP, kCx>(s, p, R, dsk, v, x3, yc + r * ystride, ch_ok);
                 }
             }
             __syncwarp();
@@ -580,7 +577,7 @@ __device__ void compute_warp(GroupSmem<NP, G> &sm, const ModalArgs &A)
     }
 }
 
-template <int NP, int G, bool kTri>
+template <int NP, int G, bool kTri, bool kCx>
 __global__ void __launch_bounds__(GroupTraits<G>::kThreads, GroupTraits<G>::kCtasPerSm)
     modal_scan_kernel(const __grid_constant__ CUtensorMap tm1, const __grid_constant__ CUtensorMap tm2,
                       const __grid_constant__ CUtensorMap tm3, const ModalArgs A)
@@ -610,11 +607,11 @@ __global__ void __launch_bounds__(GroupTraits<G>::kThreads, GroupTraits<G>::kCta
 
     const int warp = threadIdx.x >> 5;
     if (warp == G)
-        control_warp<NP, G>(sm, A, epoch);
+        control_warp<NP, G, kCx>(sm, A, epoch);
     else if (warp == G + 1)
         producer_warp<NP, G, kTri>(sm, &tm1, &tm2, &tm3, A);
     else
-        compute_warp<NP, G, kTri>(sm, A);
+        compute_warp<NP, G, kTri, kCx>(sm, A);
 
     // Every chunk the producer issued belongs to a group the compute warps
     // consumed in full, so no TMA is in flight here.
@@ -651,7 +648,41 @@ __global__ void modal_synth_kernel(const ModalSynthArgs S)
     if (n == 0) S.coef[2 * NP * row + c] = (c < S.D && S.Dskip != nullptr) ? S.Dskip[c] : 0.f;
 }
 
-template <int NP, int G, bool kTri>
+// Complex modes: slot pairs (2m, 2m+1) of mode m.  The pole is copied as
+// given; the residue slot pair holds (Re R, -Im R), so that the output sum
+// over slots is Re(R s); p^MT is formed by MT = 2^7 complex squarings in fp32,
+// (x + iy)^2 = (x x - y y) + i (2x) y.  Padded slot pairs are zero.
+template <int NP>
+__global__ void modal_csynth_kernel(const ModalSynthArgs S)
+{
+    static_assert(MT == 128, "p^MT by seven squarings");
+    const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= NP * S.Dp) return;
+    const int n = idx / S.Dp;
+    const int c = idx - n * S.Dp;
+    const bool valid = c < S.D && n < S.N;  // S.N counts slots (2 per mode)
+    const size_t row = static_cast<size_t>(S.Dp);
+    const float *pc = S.log_poles + static_cast<size_t>(c) * S.N;  // complex poles [D][N/2][2]
+    float re = 0.f, im = 0.f, r = 0.f, pn = 0.f;
+    if (valid) {
+        re = pc[n & ~1];
+        im = pc[n | 1];
+        pn = pc[n];
+        r = S.residues[static_cast<size_t>(c) * S.N + n];
+        for (int k = 0; k < 7; ++k) {
+            const float sq_re = __fmaf_rn(re, re, -__fmul_rn(im, im));
+            const float sq_im = __fmul_rn(__fadd_rn(re, re), im);
+            re = sq_re;
+            im = sq_im;
+        }
+    }
+    S.coef[n * row + c] = pn;
+    S.coef[(NP + n) * row + c] = (n & 1) ? -r : r;
+    S.coef[(2 * NP + 1 + n) * row + c] = valid ? ((n & 1) ? im : re) : 0.f;
+    if (n == 0) S.coef[2 * NP * row + c] = (c < S.D && S.Dskip != nullptr) ? S.Dskip[c] : 0.f;
+}
+
+template <int NP, int G, bool kTri, bool kCx>
 int launch_scan(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3, ModalArgs a,
                 cudaStream_t st)
 {
@@ -661,13 +692,12 @@ int launch_scan(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap 
     HYENA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
     const int smem = static_cast<int>(sizeof(GroupSmem<NP, G>));
     const int threads = GroupTraits<G>::kThreads;
+    auto kernel = modal_scan_kernel<NP, G, kTri, kCx>;
     if (configured_device != dev) {
-        HYENA_TRY(cudaFuncSetAttribute(modal_scan_kernel<NP, G, kTri>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       smem),
+        HYENA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
                   "modal scan: set max dynamic shared memory");
         HYENA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "multiprocessor count");
-        HYENA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, modal_scan_kernel<NP, G, kTri>, threads,
-                                                                smem),
+        HYENA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem),
                   "modal scan: occupancy");
         if (per_sm < 1) per_sm = 1;
         configured_device = dev;
@@ -676,17 +706,20 @@ int launch_scan(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap 
     a.nGroups = groups_per_chain * static_cast<unsigned int>(a.B) * static_cast<unsigned int>(a.nCB);
     const unsigned int slots = static_cast<unsigned int>(sms * per_sm);
     const unsigned int grid = a.nGroups < slots ? a.nGroups : slots;
-    modal_scan_kernel<NP, G, kTri><<<grid, threads, smem, st>>>(m1, m2, m3, a);
+    kernel<<<grid, threads, smem, st>>>(m1, m2, m3, a);
     HYENA_TRY(cudaGetLastError(), "modal scan launch");
     return 1;
 }
 
-template <int NP, bool kTri>
+template <int NP, bool kTri, bool kCx>
 int launch_modal_np(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3, const ModalArgs &a,
                     const ModalSynthArgs &s, cudaStream_t st)
 {
     const int total = NP * s.Dp;
-    modal_synth_kernel<NP><<<(total + 255) / 256, 256, 0, st>>>(s);
+    if (kCx)
+        modal_csynth_kernel<NP><<<(total + 255) / 256, 256, 0, st>>>(s);
+    else
+        modal_synth_kernel<NP><<<(total + 255) / 256, 256, 0, st>>>(s);
     HYENA_TRY(cudaGetLastError(), "modal synth launch");
     // Four-unit groups (two CTAs per SM) while that still gives every SM
     // several groups; two-unit groups (four CTAs per SM) for short sequences.
@@ -694,30 +727,33 @@ int launch_modal_np(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensor
     if (cudaGetDevice(&dev) == cudaSuccess) (void)cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long chains = static_cast<long long>(a.B) * a.nCB;
     const long long groups4 = chains * ((a.units + 3) / 4);
-    const int n = groups4 >= 4ll * sms ? launch_scan<NP, 4, kTri>(m1, m2, m3, a, st)
-                                       : launch_scan<NP, 2, kTri>(m1, m2, m3, a, st);
+    const int n = groups4 >= 4ll * sms ? launch_scan<NP, 4, kTri, kCx>(m1, m2, m3, a, st)
+                                       : launch_scan<NP, 2, kTri, kCx>(m1, m2, m3, a, st);
     return n < 0 ? n : n + 1;
+}
+
+template <bool kTri, bool kCx>
+int launch_modal_layout(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3, const ModalArgs &a,
+                        const ModalSynthArgs &s, int NP, cudaStream_t st)
+{
+    switch (NP) {
+        case 4: return launch_modal_np<4, kTri, kCx>(m1, m2, m3, a, s, st);
+        case 8: return launch_modal_np<8, kTri, kCx>(m1, m2, m3, a, s, st);
+        case 16: return launch_modal_np<16, kTri, kCx>(m1, m2, m3, a, s, st);
+        default: return -1;
+    }
 }
 
 }  // namespace
 
 int launch_modal(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3, ModalArgs a,
-                 const ModalSynthArgs &s, int NP, bool triples, cudaStream_t st)
+                 const ModalSynthArgs &s, int NP, bool triples, bool cx, cudaStream_t st)
 {
-    if (triples) {
-        switch (NP) {
-            case 4: return launch_modal_np<4, true>(m1, m2, m3, a, s, st);
-            case 8: return launch_modal_np<8, true>(m1, m2, m3, a, s, st);
-            case 16: return launch_modal_np<16, true>(m1, m2, m3, a, s, st);
-            default: return -1;
-        }
-    }
-    switch (NP) {
-        case 4: return launch_modal_np<4, false>(m1, m2, m3, a, s, st);
-        case 8: return launch_modal_np<8, false>(m1, m2, m3, a, s, st);
-        case 16: return launch_modal_np<16, false>(m1, m2, m3, a, s, st);
-        default: return -1;
-    }
+    if (triples)
+        return cx ? launch_modal_layout<true, true>(m1, m2, m3, a, s, NP, st)
+                  : launch_modal_layout<true, false>(m1, m2, m3, a, s, NP, st);
+    return cx ? launch_modal_layout<false, true>(m1, m2, m3, a, s, NP, st)
+              : launch_modal_layout<false, false>(m1, m2, m3, a, s, NP, st);
 }
 
 }  // namespace hyena

@@ -63,8 +63,9 @@ const char *hyena_status_string(hyena_status_t s);
 /* Version of this interface (major * 100 + minor). */
 int hyena_abi_version(void);
 
-/* Largest supported number of modes N and of FIR taps K. */
+/* Largest supported number of modes N (real; complex) and of FIR taps K. */
 #define HYENA_MAX_MODES 16
+#define HYENA_MAX_COMPLEX_MODES 8
 #define HYENA_MAX_TAPS 128
 
 /*
@@ -212,6 +213,48 @@ hyena_status_t hyena_short_decode(const hyena_bf16_t *x1, const hyena_bf16_t *x2
                                   const hyena_bf16_t *taps, const float *Dskip,
                                   hyena_bf16_t *y, int64_t ld_y,
                                   float *hist, int B, int D, int K, void *stream);
+
+/*
+ * Long modal filter with complex modes: the modal form of Evo1-1.5-7B-8K
+ * (model card, §Architecture: modal-form "poles" / "residues" kept in fp32,
+ * Hyena state size 8).  Mode n of channel c has a complex pole p and residue
+ * R, and the filter is the real part of the modal sum:
+ *
+ *   h_c[t] = Re sum_{n<N} R[c,n] p[c,n]^t,  t >= 0
+ *
+ * (a conjugate pair (p, R), (conj p, conj R) is one mode with residue 2R).
+ * poles, residues  [D, N, 2] fp32, device: (real, imaginary) of each mode.
+ *           1 <= N <= HYENA_MAX_COMPLEX_MODES.
+ * state_in, state_out  [B, D, N, 2] fp32, device, or NULL: the complex state
+ *           s_n = sum_{s<=t} p_n^(t-s) v[s] after the last token of the
+ *           previous chunk (as hyena_modal_long_conv, with complex p).
+ * workspace at least hyena_modal_long_conv_workspace_size(B, D, 2N) bytes,
+ *           zero-filled once by hyena_modal_workspace_init.
+ * Everything else, the chunking guarantees (bit-exact for chunks of whole
+ * 128-token units) and the errors are those of hyena_modal_long_conv.
+ */
+hyena_status_t hyena_modal_long_conv_complex(const hyena_bf16_t *x1, const hyena_bf16_t *x2,
+                                             const hyena_bf16_t *x3, int64_t ld_x,
+                                             const float *poles, const float *residues,
+                                             const float *Dskip,
+                                             hyena_bf16_t *y, int64_t ld_y,
+                                             const float *state_in, float *state_out,
+                                             int B, int L, int D, int N,
+                                             void *workspace, size_t workspace_bytes,
+                                             void *stream);
+
+/*
+ * One generated token through the complex-mode filter: s_n <- p_n s_n + v,
+ * y = x3 Re(sum_n R_n s_n) + Dskip v, with state [B, D, N, 2] fp32 updated in
+ * place.  Equals hyena_modal_long_conv_complex with L = 1 and
+ * state_in = state_out = state bit for bit.
+ */
+hyena_status_t hyena_modal_decode_complex(const hyena_bf16_t *x1, const hyena_bf16_t *x2,
+                                          const hyena_bf16_t *x3, int64_t ld_x,
+                                          const float *poles, const float *residues,
+                                          const float *Dskip,
+                                          hyena_bf16_t *y, int64_t ld_y,
+                                          float *state, int B, int D, int N, void *stream);
 
 /*
  * Packed projection inputs.  The Hyena input projection writes one

@@ -163,6 +163,36 @@ def test_packed_entry_points_check_their_own_arguments():
     assert lib.hyena_short_decode_packed(A, 192, 32, A, None, A + 65536, 64, None, 1, 64, 7, None) == INVALID
 
 
+def test_complex_entry_points_reject_bad_arguments():
+    lib = hy.lib()
+
+    def conv(**kw):
+        a = dict(x1=A, x2=A, x3=A, ld_x=64, p=A, r=A, ds=None, y=A + 4096, ld_y=64, s_in=None, s_out=None,
+                 B=1, L=16, D=64, N=4, ws=None, ws_bytes=0)
+        a.update(kw)
+        return lib.hyena_modal_long_conv_complex(a["x1"], a["x2"], a["x3"], a["ld_x"], a["p"], a["r"], a["ds"],
+                                                 a["y"], a["ld_y"], a["s_in"], a["s_out"], a["B"], a["L"],
+                                                 a["D"], a["N"], a["ws"], a["ws_bytes"], None)
+
+    def dec(**kw):
+        a = dict(x1=A, x2=A, x3=A, ld_x=64, p=A, r=A, ds=None, y=A + 4096, ld_y=64, s=A, B=1, D=64, N=4)
+        a.update(kw)
+        return lib.hyena_modal_decode_complex(a["x1"], a["x2"], a["x3"], a["ld_x"], a["p"], a["r"], a["ds"],
+                                              a["y"], a["ld_y"], a["s"], a["B"], a["D"], a["N"], None)
+
+    assert conv(N=0) == INVALID
+    assert conv(N=hy.MAX_COMPLEX_MODES + 1) == UNSUP
+    assert conv(p=None) == INVALID
+    assert conv(r=A + 4) == ALIGN
+    assert conv() == WORKSPACE
+    assert conv(ws=A, ws_bytes=lib.hyena_modal_long_conv_workspace_size(1, 64, 4)) == WORKSPACE  # needs 2N slots
+    assert dec(N=0) == INVALID
+    assert dec(N=9) == UNSUP
+    assert dec(s=None) == INVALID
+    assert dec(s=A + 8) == ALIGN
+    assert dec(ld_x=32) == INVALID
+
+
 def test_other_entry_points_reject_bad_arguments():
     lib = hy.lib()
     assert lib.hyena_modal_state_init(None, 1, 64, 8, None) == INVALID

@@ -63,7 +63,7 @@ constexpr int kChunksPerGroup = 2 * kChunksPerSweep;
 
 template <int G>
 struct GroupTraits {
-    static constexpr int kRing = G >= 4 ? 4 : 3;  // chunk buffers per compute warp
+    static constexpr int kRing = G >= 4 ? 4 : 5;  // chunk buffers per compute warp
     static constexpr int kThreads = 32 * (G + 2);  // compute warps, control warp, producer warp
     static constexpr int kCtasPerSm = G >= 4 ? 2 : 3;
 };

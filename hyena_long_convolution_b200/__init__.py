@@ -27,9 +27,11 @@ __all__ = [
     "last_launch_count",
     "modal_decode",
     "modal_decode_complex",
+    "modal_decode_complex_packed",
     "modal_decode_packed",
     "modal_long_conv",
     "modal_long_conv_complex",
+    "modal_long_conv_complex_packed",
     "modal_long_conv_packed",
     "modal_state_init",
     "short_conv",
@@ -438,4 +440,48 @@ def modal_decode_complex(x1, x2, x3, poles, residues, Dskip, state, y=None, stre
     rc = lib().hyena_modal_decode_complex(_ptr(x1), _ptr(x2), _ptr(x3), ld, _ptr(poles), _ptr(residues),
                                           _ptr(Dskip), _ptr(y), ld_y, _ptr(state), B, D, N, _stream(stream))
     check("hyena_modal_decode_complex", rc)
+    return y
+
+
+def modal_long_conv_complex_packed(xp, group, poles, residues, Dskip=None, y=None, state_in=None,
+                                   state_out=None, workspace: ModalWorkspace | None = None, stream=None):
+    """``modal_long_conv_complex`` with x1, x2, x3 read from one projection
+    buffer xp in channel groups of ``group`` (see ``modal_long_conv_packed``)."""
+    torch = _torch()
+    D, N = _cpar(poles, residues)
+    B, L, ld = _packed(xp, D)
+    _f32(Dskip, (D,), "Dskip")
+    _f32(state_in, (B, D, N, 2), "state_in")
+    _f32(state_out, (B, D, N, 2), "state_out")
+    if y is None:
+        y = torch.empty((B, L, D), dtype=torch.bfloat16, device=xp.device)
+    yB, yL, yD, ld_y = _bld(y, "y")
+    if (yB, yL, yD) != (B, L, D):
+        raise ValueError("y must be [B, L, D]")
+    if workspace is None:
+        workspace = ModalWorkspace(B, D, 2 * N, device=xp.device, stream=stream)
+    rc = lib().hyena_modal_long_conv_complex_packed(_ptr(xp), ld, int(group), _ptr(poles), _ptr(residues),
+                                                    _ptr(Dskip), _ptr(y), ld_y, _ptr(state_in), _ptr(state_out),
+                                                    B, L, D, N, _ptr(workspace.buf), workspace.nbytes,
+                                                    _stream(stream))
+    check("hyena_modal_long_conv_complex_packed", rc)
+    return y
+
+
+def modal_decode_complex_packed(xp, group, poles, residues, Dskip, state, y=None, stream=None):
+    """``modal_decode_complex`` with the token's x1, x2, x3 read from one
+    projection row per batch row in channel groups of ``group``."""
+    torch = _torch()
+    D, N = _cpar(poles, residues)
+    B, _, ld = _packed(xp, D, decode=True)
+    _f32(Dskip, (D,), "Dskip")
+    _f32(state, (B, D, N, 2), "state", False)
+    if y is None:
+        y = torch.empty((B, D), dtype=torch.bfloat16, device=xp.device)
+    yB, yD, ld_y = _bd(y, "y")
+    if (yB, yD) != (B, D):
+        raise ValueError("y must be [B, D] or [B, 1, D]")
+    rc = lib().hyena_modal_decode_complex_packed(_ptr(xp), ld, int(group), _ptr(poles), _ptr(residues),
+                                                 _ptr(Dskip), _ptr(y), ld_y, _ptr(state), B, D, N, _stream(stream))
+    check("hyena_modal_decode_complex_packed", rc)
     return y

@@ -49,6 +49,9 @@ SIGNATURES = {
     "hyena_modal_long_conv_complex": (_I, [_P, _P, _P, _I64, _P, _P, _P, _P, _I64, _P, _P,
                                            _I, _I, _I, _I, _P, _SZ, _P]),
     "hyena_modal_decode_complex": (_I, [_P, _P, _P, _I64, _P, _P, _P, _P, _I64, _P, _I, _I, _I, _P]),
+    "hyena_modal_long_conv_complex_packed": (_I, [_P, _I64, _I, _P, _P, _P, _P, _I64, _P, _P,
+                                                  _I, _I, _I, _I, _P, _SZ, _P]),
+    "hyena_modal_decode_complex_packed": (_I, [_P, _I64, _I, _P, _P, _P, _P, _I64, _P, _I, _I, _I, _P]),
     "hyena_modal_state_init": (_I, [_P, _I, _I, _I, _P]),
     "hyena_workspace_check": (_I, [_P, _P]),
 }

@@ -491,6 +491,28 @@ hyena_status_t hyena_modal_decode_complex(const hyena_bf16_t *x1, const hyena_bf
                              stream, true);
 }
 
+hyena_status_t hyena_modal_long_conv_complex_packed(const hyena_bf16_t *xp, int64_t ld_x, int group,
+                                                    const float *poles, const float *residues, const float *Dskip,
+                                                    hyena_bf16_t *y, int64_t ld_y, const float *state_in,
+                                                    float *state_out, int B, int L, int D, int N, void *workspace,
+                                                    size_t workspace_bytes, void *stream)
+{
+    const hyena_status_t st = check_packed(xp, ld_x, group, y, ld_y, B, L, D);
+    if (st != HYENA_OK) return st;
+    return modal_long_conv_impl(packed_source(xp, ld_x, group), poles, residues, Dskip, y, ld_y, state_in,
+                                state_out, B, L, D, N, workspace, workspace_bytes, stream, true);
+}
+
+hyena_status_t hyena_modal_decode_complex_packed(const hyena_bf16_t *xp, int64_t ld_x, int group, const float *poles,
+                                                 const float *residues, const float *Dskip, hyena_bf16_t *y,
+                                                 int64_t ld_y, float *state, int B, int D, int N, void *stream)
+{
+    const hyena_status_t st = check_packed(xp, ld_x, group, y, ld_y, B, 1, D);
+    if (st != HYENA_OK) return st;
+    return modal_decode_impl(packed_source(xp, ld_x, group), poles, residues, Dskip, y, ld_y, state, B, D, N,
+                             stream, true);
+}
+
 hyena_status_t hyena_short_decode(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
                                   int64_t ld_x, const hyena_bf16_t *taps, const float *Dskip, hyena_bf16_t *y,
                                   int64_t ld_y, float *hist, int B, int D, int K, void *stream)

@@ -307,6 +307,23 @@ hyena_status_t hyena_short_decode_packed(const hyena_bf16_t *xp, int64_t ld_x, i
                                          hyena_bf16_t *y, int64_t ld_y,
                                          float *hist, int B, int D, int K, void *stream);
 
+/* The complex-mode filter (hyena_modal_long_conv_complex, hyena_modal_decode_complex)
+ * with packed projection inputs, as above. */
+hyena_status_t hyena_modal_long_conv_complex_packed(const hyena_bf16_t *xp, int64_t ld_x, int group,
+                                                    const float *poles, const float *residues,
+                                                    const float *Dskip,
+                                                    hyena_bf16_t *y, int64_t ld_y,
+                                                    const float *state_in, float *state_out,
+                                                    int B, int L, int D, int N,
+                                                    void *workspace, size_t workspace_bytes,
+                                                    void *stream);
+
+hyena_status_t hyena_modal_decode_complex_packed(const hyena_bf16_t *xp, int64_t ld_x, int group,
+                                                 const float *poles, const float *residues,
+                                                 const float *Dskip,
+                                                 hyena_bf16_t *y, int64_t ld_y,
+                                                 float *state, int B, int D, int N, void *stream);
+
 /*
  * Zero-fills a modal state [B, D, N] fp32 (the state before the first token
  * of a sequence): the start of chunked prefill.

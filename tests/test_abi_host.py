@@ -134,6 +134,9 @@ def packed_calls(lib, xp=A, ld_x=192, group=1, y=A + 65536, ld_y=64, B=1, L=16, 
         "fir": lib.hyena_short_conv_packed(xp, ld_x, group, A, None, y, ld_y, None, None, B, L, D, 7, None),
         "mdec": lib.hyena_modal_decode_packed(xp, ld_x, group, A, A, None, y, ld_y, A, B, D, 8, None),
         "fdec": lib.hyena_short_decode_packed(xp, ld_x, group, A, None, y, ld_y, A, B, D, 7, None),
+        "cmodal": lib.hyena_modal_long_conv_complex_packed(xp, ld_x, group, A, A, None, y, ld_y, None, None,
+                                                           B, L, D, 4, None, 0, None),
+        "cdec": lib.hyena_modal_decode_complex_packed(xp, ld_x, group, A, A, None, y, ld_y, A, B, D, 4, None),
     }
 
 

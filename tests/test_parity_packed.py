@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 
 import oracle
-from synth import make_fir_inputs, make_modal_inputs
+from synth import make_cmodal_inputs, make_fir_inputs, make_modal_inputs
 
 from .helpers import assert_close, bits_of, from_dev_bf16, metrics, to_dev_bf16, to_dev_f32
 
@@ -167,3 +167,33 @@ def test_decode_packed(group):
     torch.cuda.synchronize()
     assert np.array_equal(bits_of(yf), bits_of(yfq))
     assert torch.equal(H1, H2)
+
+
+@pytest.mark.parametrize("group", [1, 64])
+def test_complex_modes_packed(group):
+    """Complex modes from a packed buffer: bit-equal to the plain complex call,
+    prefill and decode."""
+    import torch
+    import hyena_long_convolution_b200 as hy
+    B, L, D, N = 2, 300, 128, 8
+    inp = make_cmodal_inputs(B, L, D, N, seed=17 + group)
+    p, R, Ds = to_dev_f32(inp["poles"]), to_dev_f32(inp["residues"]), to_dev_f32(inp["Dskip"])
+    xp = dev_packed(inp, group, ld_pad=8)
+    S0 = torch.randn((B, D, N, 2), device="cuda")
+    S1, S2 = torch.empty_like(S0), torch.empty_like(S0)
+    y = hy.modal_long_conv_complex_packed(xp, group, p, R, Ds, state_in=S0, state_out=S1)
+    xs = [to_dev_bf16(inp[k]) for k in ("x1", "x2", "x3")]
+    yq = hy.modal_long_conv_complex(*xs, p, R, Ds, state_in=S0, state_out=S2)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits_of(y), bits_of(yq))
+    assert torch.equal(S1, S2)
+    ref_y, _ = oracle.cmodal_recurrence(inp["x1"], inp["x2"], inp["x3"], inp["poles"], inp["residues"],
+                                        inp["Dskip"], S0.cpu().numpy().astype(np.float64))
+    assert_close(from_dev_bf16(y), ref_y, "complex packed y")
+    # one decode step from the packed buffer's first row
+    S3, S4 = S0.clone(), S0.clone()
+    yd = hy.modal_decode_complex_packed(xp[:, 0], group, p, R, Ds, S3)
+    ydq = hy.modal_decode_complex(*(x[:, 0] for x in xs), p, R, Ds, S4)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits_of(yd), bits_of(ydq))
+    assert torch.equal(S3, S4)

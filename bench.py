@@ -161,6 +161,24 @@ def dist_env():
     return world, rank, local
 
 
+def max_over_ranks(pg, values, device):
+    """Element-wise maximum over all ranks of per-rank timings (the slowest
+    replica bounds the job); the values themselves without a process group.
+    Every rank calls it at the same point with the same number of values."""
+    if pg is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_rate(world, units_per_step, steps, total_ms):
+    """Whole-job throughput: the units every rank processed over the slowest
+    rank's time."""
+    return world * units_per_step * steps / (total_ms / 1e3)
+
+
 # ------------------------------------------------------------------ clocks
 
 
@@ -531,24 +549,15 @@ def run_gpu(args, wl):
         per = time_steps(step, args.steps, 0, device)
         clk.mark("end")
     barrier()
-    t_total_ms = sum(per)
+    t_total_ms = max_over_ranks(pg, [sum(per)], device)[0]
     ms_step = t_total_ms / args.steps
-    if pg is not None:
-        t = torch.tensor([t_total_ms], device=device)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        t_total_ms = float(t.item())
-        ms_step = t_total_ms / args.steps
-    value = world * chtok * args.steps / (t_total_ms / 1e3)
+    value = job_rate(world, chtok, args.steps, t_total_ms)
 
     # e2e through the binding with host buffers (fewer steps: PCIe-bound)
     e_steps = max(3, min(args.steps, 5))
     eper, h2d, d2h = e2e_leg(wl, host, dev, device, e_steps, 3)
-    e_total = sum(eper)
-    if pg is not None:
-        t = torch.tensor([e_total], device=device)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e_total = float(t.item())
-    e_value = world * chtok * e_steps / (e_total / 1e3)
+    e_total = max_over_ranks(pg, [sum(eper)], device)[0]
+    e_value = job_rate(world, chtok, e_steps, e_total)
 
     peak, peak_kind = measured_peaks()
     per_sorted = sorted(per)

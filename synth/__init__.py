@@ -6,11 +6,11 @@ operator's arithmetic, so both the fp64 oracle and the CUDA library can be fed
 from it without sharing any code with each other.
 """
 from .inputs import (  # noqa: F401
-    CONFIGS,
+    WORKLOAD_SHAPES,
     bf16_bits_to_f32,
     f32_to_bf16_bits,
     make_cmodal_inputs,
     make_fir_inputs,
-    make_inputs_for_config,
+    make_workload_inputs,
     make_modal_inputs,
 )

@@ -38,19 +38,19 @@ import numpy as np
 
 ROW_BLOCK = 1024
 
-# The five workloads: shapes and distributions as the library's acceptance
-# configurations define them.
-CONFIGS = {
-    0: dict(kind="modal", B=1, L=1024, D=64, N=8, seed=0, wide_range=False,
-            name="modal B1 L1024 D64 N8"),
-    1: dict(kind="fir", B=2, L=8192, D=4096, K=(7, 128), seed=1,
-            name="short FIR B2 L8192 D4096 K7/K128"),
-    2: dict(kind="modal", B=1, L=32768, D=4096, N=16, seed=2, wide_range=False,
-            name="modal B1 L32768 D4096 N16"),
-    3: dict(kind="modal", B=1, L=131072, D=4096, N=16, seed=3, wide_range=False,
-            chunk=1024, name="modal B1 L131072 D4096 N16, 128 chunks of 1024"),
-    4: dict(kind="modal", B=1, L=262144, D=4096, N=16, seed=4, wide_range=True,
-            name="modal B1 L262144 D4096 N16, wide dynamic range"),
+# The five acceptance workloads, by name: shapes and distributions; each
+# name's seed is fixed here and used for every draw of that workload.
+WORKLOAD_SHAPES = {
+    "modal_1k": dict(kind="modal", B=1, L=1024, D=64, N=8, seed=0, wide_range=False,
+                     name="modal B1 L1024 D64 N8"),
+    "fir_8k": dict(kind="fir", B=2, L=8192, D=4096, K=(7, 128), seed=1,
+                   name="short FIR B2 L8192 D4096 K7/K128"),
+    "modal_32k": dict(kind="modal", B=1, L=32768, D=4096, N=16, seed=2, wide_range=False,
+                      name="modal B1 L32768 D4096 N16"),
+    "modal_131k_chunked": dict(kind="modal", B=1, L=131072, D=4096, N=16, seed=3, wide_range=False,
+                               chunk=1024, name="modal B1 L131072 D4096 N16, 128 chunks of 1024"),
+    "modal_262k_wide": dict(kind="modal", B=1, L=262144, D=4096, N=16, seed=4, wide_range=True,
+                            name="modal B1 L262144 D4096 N16, wide dynamic range"),
 }
 
 
@@ -157,8 +157,8 @@ def make_fir_inputs(B: int, L: int, D: int, K: int, seed: int, with_skip: bool =
     return dict(x1=x1, x2=x2, x3=x3, taps=taps, Dskip=Dskip, B=B, L=L, D=D, K=K)
 
 
-def make_inputs_for_config(idx: int, K: int | None = None, threads: int | None = None) -> dict:
-    cfg = CONFIGS[idx]
+def make_workload_inputs(name: str, K: int | None = None, threads: int | None = None) -> dict:
+    cfg = WORKLOAD_SHAPES[name]
     if cfg["kind"] == "fir":
         K = cfg["K"][0] if K is None else K
         return make_fir_inputs(cfg["B"], cfg["L"], cfg["D"], K, cfg["seed"], threads=threads)

@@ -45,7 +45,7 @@ def small_modal(B=2, L=96, D=12, N=5, seed=11, with_state=True):
 # ---------------------------------------------------------------- modal form
 
 
-def test_direct_equals_recurrence_config0_shape():
+def test_direct_equals_recurrence_modal_1k_shape():
     # Two independently coded forms of the same filter (O(L^2) convolution with
     # the synthesised h, versus one recurrence per mode).
     inp = make_modal_inputs(1, 1024, 64, 8, 0, threads=1)

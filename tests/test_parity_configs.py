@@ -1,8 +1,9 @@
 """Parity at the five acceptance workloads' full sizes, in the launch
 configuration the benchmark times.
 
-Config 0 and config 2 are compared element by element with the fp64 oracle
-over the whole output tensor.  For the 131K- and 262K-token workloads the
+The 1K- and 32K-token modal workloads (and both FIR workloads, in their own
+files) are compared element by element with the fp64 oracle over the whole
+output tensor.  For the 131K- and 262K-token workloads the
 oracle runs on a sample of channels (every position of those channels), and
 the whole tensor is checked through properties that hold at any size:
 chunked feeding in whole 128-token units reproduces the single pass bit for
@@ -12,7 +13,7 @@ import numpy as np
 import pytest
 
 import oracle
-from synth import CONFIGS, make_inputs_for_config
+from synth import WORKLOAD_SHAPES, make_workload_inputs
 
 from .helpers import assert_close, bits_of, from_dev_bf16, metrics, to_dev_bf16, to_dev_f32
 
@@ -58,47 +59,47 @@ def sampled_oracle(inp, chans):
                                    inp["residues"][chans], inp["Dskip"][chans])
 
 
-def test_config2_full_tensor():
+def test_modal_32k_full_tensor():
     import torch
-    inp = make_inputs_for_config(2)
+    inp = make_workload_inputs("modal_32k")
     dev = Dev(inp)
     y, S = modal_run(dev, inp)
     ref_y, ref_S = oracle.modal_recurrence(inp["x1"], inp["x2"], inp["x3"], inp["log_poles"],
                                            inp["residues"], inp["Dskip"])
-    assert_close(from_dev_bf16(y), ref_y, "config 2")
+    assert_close(from_dev_bf16(y), ref_y, "modal 32K")
     rel, _ = metrics(S.cpu().numpy().astype(np.float64), ref_S)
     assert rel < 1e-4
     del y
     torch.cuda.empty_cache()
 
 
-def test_config3_chunked_prefill():
+def test_modal_131k_chunked_prefill():
     import torch
-    inp = make_inputs_for_config(3)
+    inp = make_workload_inputs("modal_131k_chunked")
     dev = Dev(inp)
     y1, S1 = modal_run(dev, inp)
-    yc, Sc = modal_run(dev, inp, chunk=CONFIGS[3]["chunk"])
+    yc, Sc = modal_run(dev, inp, chunk=WORKLOAD_SHAPES["modal_131k_chunked"]["chunk"])
     # 1024-token chunks are whole 128-token units: bitwise equal to the single pass
     assert torch.equal(yc.view(torch.int16), y1.view(torch.int16))
     assert torch.equal(Sc, S1)
     chans = sample_channels(inp["D"], seed=3)
     ref_y, ref_S = sampled_oracle(inp, chans)
     idx = torch.from_numpy(chans).cuda()
-    assert_close(from_dev_bf16(yc.index_select(2, idx)), ref_y, "config 3 (sampled channels)")
+    assert_close(from_dev_bf16(yc.index_select(2, idx)), ref_y, "modal 131K in 1024-token chunks (sampled channels)")
     rel, _ = metrics(Sc[:, chans].cpu().numpy().astype(np.float64), ref_S)
     assert rel < 1e-4
 
 
-def test_config4_long_context_wide_range():
+def test_modal_262k_long_context_wide_range():
     import torch
-    inp = make_inputs_for_config(4)
+    inp = make_workload_inputs("modal_262k_wide")
     dev = Dev(inp)
     y1, S1 = modal_run(dev, inp)
     assert bool(torch.isfinite(y1.float()).all())
     chans = sample_channels(inp["D"], seed=4)
     ref_y, ref_S = sampled_oracle(inp, chans)
     idx = torch.from_numpy(chans).cuda()
-    assert_close(from_dev_bf16(y1.index_select(2, idx)), ref_y, "config 4 single pass", per_channel=True)
+    assert_close(from_dev_bf16(y1.index_select(2, idx)), ref_y, "modal 262K single pass", per_channel=True)
     rel, _ = metrics(S1[:, chans].cpu().numpy().astype(np.float64), ref_S)
     assert rel < 1e-4
     y1_bits = bits_of(y1.index_select(2, idx))

@@ -3,7 +3,7 @@ import numpy as np
 import pytest
 
 import oracle
-from synth import CONFIGS, make_fir_inputs
+from synth import WORKLOAD_SHAPES, make_fir_inputs
 
 from .helpers import assert_close, bits_of, from_dev_bf16, metrics, to_dev_bf16, to_dev_f32
 
@@ -83,10 +83,10 @@ def test_chunked_is_bitwise_single_pass(K, chunks):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("K", list(CONFIGS[1]["K"]))
-def test_config1_full_size(K):
+@pytest.mark.parametrize("K", list(WORKLOAD_SHAPES["fir_8k"]["K"]))
+def test_fir_8k_full_size(K):
     import torch
-    c = CONFIGS[1]
+    c = WORKLOAD_SHAPES["fir_8k"]
     inp = make_fir_inputs(c["B"], c["L"], c["D"], K, c["seed"])
     y, _ = run_gpu(inp)
     rng = np.random.default_rng(K)
@@ -94,5 +94,5 @@ def test_config1_full_size(K):
     sub = {k: np.ascontiguousarray(inp[k][:, :, chans]) for k in ("x1", "x2", "x3")}
     ref, _ = oracle.fir(sub["x1"], sub["x2"], sub["x3"], inp["taps"][chans], None, None)
     idx = torch.from_numpy(chans).cuda()
-    assert_close(from_dev_bf16(y.index_select(2, idx)), ref, f"config 1 K={K}")
+    assert_close(from_dev_bf16(y.index_select(2, idx)), ref, f"FIR 8K K={K}")
     assert bool(torch.isfinite(y.float()).all())

@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 
 import oracle
-from synth import CONFIGS, make_modal_inputs
+from synth import WORKLOAD_SHAPES, make_modal_inputs
 
 from .helpers import assert_close, bits_of, from_dev_bf16, metrics, to_dev_bf16, to_dev_f32
 
@@ -59,14 +59,14 @@ def check(inp, state_in=None, **kw):
     return y, S
 
 
-def test_config0_full():
-    c = CONFIGS[0]
+def test_modal_1k_full():
+    c = WORKLOAD_SHAPES["modal_1k"]
     inp = make_modal_inputs(c["B"], c["L"], c["D"], c["N"], c["seed"])
     check(inp)
 
 
-def test_config0_with_state_and_direct_form():
-    c = CONFIGS[0]
+def test_modal_1k_with_state_and_direct_form():
+    c = WORKLOAD_SHAPES["modal_1k"]
     inp = make_modal_inputs(c["B"], c["L"], c["D"], c["N"], c["seed"])
     S = np.random.default_rng(1).standard_normal((1, 64, 8))
     y, _ = check(inp, S)

@@ -365,6 +365,145 @@ __global__ void __launch_bounds__(FW * 32)
     }
 }
 
+// Short filters (K <= 8, halo of at most 8 rows): the window values are formed
+// from the bf16 x1, x2 rows as they are used instead of from an fp32 v buffer,
+// and each warp computes its 16 outputs in two halves of 8.  That keeps the CTA
+// at 53 KB of shared memory and at most 64 registers, four CTAs per SM
+// instead of two, for this HBM-bound case.  kTri: the rows are the interleaved
+// per-channel triples (96 words per row), read the same way.  The FMA order per
+// output is the general kernel's (taps in lag order from a zero accumulator),
+// so results are bit-identical to it.
+constexpr int kSmallMaxK = 8;
+constexpr int kSmallHalf = 8;  // outputs per pass
+
+__host__ __device__ inline size_t fir_small_smem_bytes(int HR, int K, bool tri)
+{
+    const size_t rows = static_cast<size_t>(HR) + FT;
+    const size_t x = tri ? rows * 3 * kRowWords * 4 : rows * kRowWords * 4 * 2 + static_cast<size_t>(FT) * kRowWords * 4;
+    return x + static_cast<size_t>(K) * 32 * 8 + 16;
+}
+
+template <bool kTri>
+__global__ void __launch_bounds__(FW * 32, 4)
+    fir_small_kernel(const __grid_constant__ CUtensorMap tm1, const __grid_constant__ CUtensorMap tm2,
+                     const __grid_constant__ CUtensorMap tm3, const __grid_constant__ CUtensorMap th1,
+                     const __grid_constant__ CUtensorMap th2, const FirArgs A)
+{
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const int HR = A.HR, K = A.K, H = K - 1;
+    const int rows = HR + FT;
+    uint32_t *x1 = reinterpret_cast<uint32_t *>(smem_raw);  // kTri: the interleaved rows
+    uint32_t *x2 = x1 + rows * kRowWords;
+    uint32_t *x3 = x2 + rows * kRowWords;
+    float2 *taps = reinterpret_cast<float2 *>(kTri ? x1 + rows * 3 * kRowWords : x3 + FT * kRowWords);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(taps + K * 32);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int cb = blockIdx.x;
+    const int t0 = blockIdx.y * FT;
+    const int b = blockIdx.z;
+    const int c0 = cb * FCH + 2 * lane;
+    const bool ch_ok = c0 < A.D;
+
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        const int ch = cb * FCH;
+        if constexpr (kTri) {
+            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows * 3 * kRowWords * 4));
+            if (HR > 0) tma_load_4d(x1, &th1, bar, 3 * ch, 0, t0 - HR, b);
+            tma_load_4d(x1 + HR * 3 * kRowWords, &tm1, bar, 3 * ch, 0, t0, b);
+        } else {
+            const int cx = ch % A.group, cg = ch / A.group;
+            mbar_arrive_expect_tx(bar, static_cast<uint32_t>((2 * rows + FT) * kRowWords * 4));
+            if (HR > 0) {
+                tma_load_4d(x1, &th1, bar, cx, cg, t0 - HR, b);
+                tma_load_4d(x2, &th2, bar, cx, cg, t0 - HR, b);
+            }
+            tma_load_4d(x1 + HR * kRowWords, &tm1, bar, cx, cg, t0, b);
+            tma_load_4d(x2 + HR * kRowWords, &tm2, bar, cx, cg, t0, b);
+            tma_load_4d(x3, &tm3, bar, cx, cg, t0, b);
+        }
+    }
+    for (int idx = tid; idx < K * 32; idx += FW * 32) {
+        const int k = idx >> 5, l = idx & 31;
+        const int c = cb * FCH + 2 * l;
+        float2 t = make_float2(0.f, 0.f);
+        if (c < A.D) {
+            t.x = __uint_as_float(static_cast<uint32_t>(A.taps[static_cast<size_t>(c) * K + k]) << 16);
+            t.y = __uint_as_float(static_cast<uint32_t>(A.taps[static_cast<size_t>(c + 1) * K + k]) << 16);
+        }
+        taps[idx] = t;
+    }
+    const bool ok = mbar_wait_bounded(bar, 0);
+    if (__syncthreads_or(!ok)) {
+        (void)mbar_wait_bounded(bar, 0);
+        return;  // tiles never arrived; output left unwritten
+    }
+
+    // v of row r (rows before t = 0 from hist_in, or zero)
+    auto vrow = [&](int r) {
+        const int t = t0 - HR + r;
+        if (t >= 0) {
+            if constexpr (kTri) {
+                const uint32_t *rw = x1 + r * 3 * kRowWords + 3 * lane;
+                const uint32_t w0 = rw[0], w1 = rw[1], w2 = rw[2];
+                return __fmul2_rn(tri_x1(w0, w1), tri_x2(w0, w2));
+            } else {
+                return __fmul2_rn(bf16x2_to_float2(x1[r * kRowWords + lane]),
+                                  bf16x2_to_float2(x2[r * kRowWords + lane]));
+            }
+        }
+        if (t >= -H && A.hist_in != nullptr && ch_ok)
+            return *reinterpret_cast<const float2 *>(A.hist_in + (static_cast<size_t>(b) * H + (H + t)) * A.D + c0);
+        return make_float2(0.f, 0.f);
+    };
+    const float2 dsk = (A.Dskip != nullptr && ch_ok) ? make_float2(A.Dskip[c0], A.Dskip[c0 + 1])
+                                                     : make_float2(0.f, 0.f);
+    const size_t ystride = static_cast<size_t>(A.ld_y) / 2;
+#pragma unroll 1
+    for (int h = 0; h < FRW / kSmallHalf; ++h) {
+        const int orow = warp * FRW + h * kSmallHalf;  // first output row of this pass (tile-relative)
+        const int row0 = HR + orow;                    // its v row
+        float2 acc[kSmallHalf];
+#pragma unroll
+        for (int i = 0; i < kSmallHalf; ++i) acc[i] = make_float2(0.f, 0.f);
+        // window rows row0 - (kSmallMaxK - 1) .. row0 + kSmallHalf - 1 (only the last K - 1 + 8 are used)
+        float2 w[kSmallHalf + kSmallMaxK - 1];
+#pragma unroll
+        for (int j = 0; j < kSmallHalf + kSmallMaxK - 1; ++j) {
+            const int r = row0 - (kSmallMaxK - 1) + j;
+            w[j] = r >= 0 ? vrow(r) : make_float2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int q = 0; q < kSmallMaxK; ++q) {
+            if (q < K) {
+                const float2 tq = taps[q * 32 + lane];
+#pragma unroll
+                for (int i = 0; i < kSmallHalf; ++i) acc[i] = __ffma2_rn(tq, w[i - q + kSmallMaxK - 1], acc[i]);
+            }
+        }
+        const int tw0 = t0 + orow;
+        const int nvalid = min(kSmallHalf, A.L - tw0);
+        uint32_t *yrow = reinterpret_cast<uint32_t *>(A.y + (static_cast<size_t>(b) * A.L + tw0) * A.ld_y + c0);
+#pragma unroll
+        for (int i = 0; i < kSmallHalf; ++i) {
+            if (i < nvalid && ch_ok) {
+                float2 x3v;
+                if constexpr (kTri) {
+                    const uint32_t *rw = x1 + (HR + orow + i) * 3 * kRowWords + 3 * lane;
+                    x3v = tri_x3(rw[1], rw[2]);
+                } else {
+                    x3v = bf16x2_to_float2(x3[(orow + i) * kRowWords + lane]);
+                }
+                yrow[i * ystride] = float2_to_bf16x2(__ffma2_rn(dsk, w[i + kSmallMaxK - 1], __fmul2_rn(x3v, acc[i])));
+            }
+        }
+    }
+}
+
 // hist_out[b][j][c] = v[L-H+j] (from hist_in when that index is negative).
 // One thread per (batch row, channel pair) walks j upward, so reading
 // hist_in[j + L] before writing hist_out[j + L] keeps in-place use safe.
@@ -403,8 +542,9 @@ int launch_fir(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &
 {
     int launches = 0;
     if (a.L > 0) {
+        const bool small = a.K <= kSmallMaxK;
         const int mode = triples ? kTriples : (fir_in_place(a.HR, a.K) ? kInPlace : kSeparate);
-        const size_t smem = fir_smem_bytes(a.HR, a.K, mode);
+        const size_t smem = small ? fir_small_smem_bytes(a.HR, a.K, triples) : fir_smem_bytes(a.HR, a.K, mode);
         static int configured_device = -1;
         int dev = 0;
         HYENA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
@@ -419,10 +559,22 @@ int launch_fir(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &
             HYENA_TRY(cudaFuncSetAttribute(fir_kernel<kTriples>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(fir_smem_bytes(kMaxHalo, HYENA_MAX_TAPS, kTriples))),
                       "fir: set max dynamic shared memory");
+            HYENA_TRY(cudaFuncSetAttribute(fir_small_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(fir_small_smem_bytes(fir_halo_rows(kSmallMaxK),
+                                                                                 kSmallMaxK, false))),
+                      "fir: set max dynamic shared memory");
+            HYENA_TRY(cudaFuncSetAttribute(fir_small_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(fir_small_smem_bytes(fir_halo_rows(kSmallMaxK),
+                                                                                 kSmallMaxK, true))),
+                      "fir: set max dynamic shared memory");
             configured_device = dev;
         }
         const dim3 grid((a.D + FCH - 1) / FCH, (a.L + FT - 1) / FT, a.B);
-        if (mode == kTriples)
+        if (small && triples)
+            fir_small_kernel<true><<<grid, FW * 32, smem, st>>>(m1, m2, m3, h1, h2, a);
+        else if (small)
+            fir_small_kernel<false><<<grid, FW * 32, smem, st>>>(m1, m2, m3, h1, h2, a);
+        else if (mode == kTriples)
             fir_kernel<kTriples><<<grid, FW * 32, smem, st>>>(m1, m2, m3, h1, h2, a);
         else if (mode == kInPlace)
             fir_kernel<kInPlace><<<grid, FW * 32, smem, st>>>(m1, m2, m3, h1, h2, a);

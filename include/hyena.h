@@ -16,16 +16,21 @@
  * FIR window (hcs/hcm) is carried from one call to the next, and every
  * position of every chunk is produced (Evo2-7B-262K model card, "Custom
  * cache"; turboquant-evo2-int4 model card, §"Important: a correctness fix
- * comes with this" and §"Chunk size").
+ * comes with this" and §"Chunk size").  The long filter is also offered with
+ * complex modes, the modal form of Evo 1 (h_c[t] = Re sum_n R p^t), and every
+ * operation can read x1, x2, x3 straight from one packed in_proj output
+ * (*_packed entry points).
  *
  * Conventions shared by every entry point
  *   - Tensors are bf16 (passed as hyena_bf16_t bit patterns), layout
  *     [B, L, D], channel-contiguous: element (b, t, c) sits at
  *     (b * L + t) * ld + c.  ld >= D is a row stride in elements, so x1, x2,
  *     x3 may be three views of one [B, L, 3D] projection output (ld = 3D).
- *   - Every device pointer is a device address owned by the caller; the
- *     library allocates no device memory.  Pointers must be 16-byte aligned,
- *     D and ld must be multiples of 8.
+ *   - Every device pointer is a device address owned by the caller; no
+ *     entry point allocates device memory (the modal conv takes a caller
+ *     workspace; its allocation-free variant uses a fixed array of the
+ *     library's module).  Pointers must be 16-byte aligned, D and ld must be
+ *     multiples of 8.
  *   - Arithmetic is fp32 (v is exact in fp32); y is rounded once to bf16
  *     (round to nearest even).  NaN and Inf propagate.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy

@@ -11,6 +11,7 @@ dropped cross term or an off-by-one power fails at least one of them.
 """
 import cmath
 import math
+import os
 
 import numpy as np
 import pytest
@@ -152,3 +153,27 @@ def test_skip_sits_outside_the_gate():
                                     np.zeros_like(inp["residues"]), inp["Dskip"])
     v = bf16_bits_to_f32(inp["x1"]).astype(np.float64) * bf16_bits_to_f32(inp["x2"])
     np.testing.assert_array_equal(y, inp["Dskip"][None, None, :].astype(np.float64) * v)
+
+
+def test_golden_quarter_turn():
+    """Hand-derived fixture tests/golden/cmodal_quarter_turn.txt (derivation in
+    its header): both oracle forms reproduce the exact dyadic values."""
+    g = {}
+    with open(os.path.join(os.path.dirname(__file__), "golden", "cmodal_quarter_turn.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                k, *vals = line.split()
+                g[k] = [float(v) for v in vals]
+    L, N = int(g["L"][0]), int(g["N"][0])
+    sh = (1, L, 1)
+    x = [bits(np.array(g[k], np.float32).reshape(sh)) for k in ("x1", "x2", "x3")]
+    p = np.array(g["poles"], np.float32).reshape(1, N, 2)
+    R = np.array(g["residues"], np.float32).reshape(1, N, 2)
+    Ds = np.array(g["Dskip"], np.float32)
+    S = np.array(g["state_in"]).reshape(1, 1, N, 2)
+    tol = g["tol"][0]
+    for fn in (oracle.cmodal_recurrence, oracle.cmodal_direct):
+        y, s = fn(*x, p, R, Ds, S)
+        np.testing.assert_allclose(y.ravel(), g["y"], rtol=tol, atol=tol)
+        np.testing.assert_allclose(s.ravel(), g["state_out"], rtol=tol, atol=tol)

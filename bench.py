@@ -161,6 +161,16 @@ def dist_env():
     return world, rank, local
 
 
+def workload_config(wl):
+    """The workload part of the JSON line's config (shared by both arms)."""
+    return {"workload": wl["desc"], "B": wl["B"], "L": wl["L"], "D": wl["D"],
+            **({"N": wl["N"], "modes": "complex" if wl.get("cx") else "real"} if wl["kind"] == "modal"
+               else {"K": wl["K"]}),
+            "mode": "decode (one-token calls)" if wl.get("decode") else "prefill",
+            "input_layout": (f"packed projection, channel groups of {wl['group']}" if wl.get("group")
+                             else "three [B, L, D] tensors")}
+
+
 def max_over_ranks(pg, values, device):
     """Element-wise maximum over all ranks of per-rank timings (the slowest
     replica bounds the job); the values themselves without a process group.
@@ -594,12 +604,7 @@ def run_gpu(args, wl):
         "dtype": "f32",
         "io_dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 inputs, pages' shapes)",
-        "config": {"workload": wl["desc"], "B": wl["B"], "L": wl["L"], "D": wl["D"],
-                   **({"N": wl["N"], "modes": "complex" if wl.get("cx") else "real"} if wl["kind"] == "modal"
-                      else {"K": wl["K"]}),
-                   "mode": "decode (one-token calls)" if wl.get("decode") else "prefill",
-                   "input_layout": (f"packed projection, channel groups of {wl['group']}" if wl.get("group")
-                                    else "three [B, L, D] tensors"),
+        "config": {**workload_config(wl),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "cache": "inputs larger than L2 (no flush)", "graph": bool(args.graph)},
         "roofline": roof,
@@ -637,7 +642,7 @@ def run_reference(args, wl):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": chtok / value * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl["desc"], "B": wl["B"], "L": wl["L"], "D": wl["D"]},
+        "config": {**workload_config(wl), "parallelism": "host cores (fp64 oracle)"},
         "impl": "reference",
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": f"per step: {sample}"},

@@ -14,6 +14,9 @@ stride ld >= D is allowed, so x1, x2, x3 may be views of one [B, L, 3D]
 projection output.  The ``*_packed`` variants read the three inputs from one
 [B, L, >= 3D] projection buffer whose rows hold channel groups of ``group``
 channels as [x1 | x2 | x3] (group = 1: per-channel triples x1_c x2_c x3_c).
+The ``*_complex`` variants take complex modes (poles and residues as [D, N, 2]
+fp32 pairs; h_c[t] = Re sum_n R p^t), and the ``*_decode`` functions advance
+the modal state or the FIR window by one generated token.
 """
 from __future__ import annotations
 

@@ -177,3 +177,25 @@ def test_golden_quarter_turn():
         y, s = fn(*x, p, R, Ds, S)
         np.testing.assert_allclose(y.ravel(), g["y"], rtol=tol, atol=tol)
         np.testing.assert_allclose(s.ravel(), g["state_out"], rtol=tol, atol=tol)
+
+
+@pytest.mark.parametrize("omega", [math.pi / 2, math.pi])
+def test_steady_state_frequency_response(omega):
+    # h[k] = Re sum R p^k has the real transfer function
+    # H(z) = 1/2 sum_n [R_n / (1 - p_n z^-1) + conj(R_n) / (1 - conj(p_n) z^-1)];
+    # for v[t] = cos(omega t) the steady state is Re(H(e^{j omega}) e^{j omega t}).
+    L, D, N = 600, 3, 3
+    g = np.random.default_rng(9)
+    rho = g.uniform(0.05, 0.9, (D, N))
+    th = g.uniform(0.0, math.pi, (D, N))
+    poles = np.stack([rho * np.cos(th), rho * np.sin(th)], -1).astype(np.float32)
+    res = g.standard_normal((D, N, 2)).astype(np.float32)
+    t = np.arange(L)
+    x1 = np.round(np.cos(omega * t)).astype(np.float32)[None, :, None].repeat(D, 2)  # exactly 1, 0, -1
+    y, _ = oracle.cmodal_recurrence(bits(x1), ones_bits((1, L, D)), ones_bits((1, L, D)), poles, res)
+    z1 = np.exp(-1j * omega)
+    for c in range(D):
+        P, R = cx(poles[c]), cx(res[c])
+        H = 0.5 * np.sum(R / (1.0 - P * z1) + np.conj(R) / (1.0 - np.conj(P) * z1))
+        ref = np.real(H * np.exp(1j * omega * t))
+        np.testing.assert_allclose(y[0, 300:, c], ref[300:], rtol=1e-10, atol=1e-10)

@@ -120,6 +120,25 @@ def test_each_mode_matches_scipy_lfilter():
         np.testing.assert_allclose(y[0, :, c], ref, rtol=1e-11, atol=1e-11)
 
 
+@pytest.mark.parametrize("omega", [math.pi / 2, math.pi])
+def test_steady_state_frequency_response(omega):
+    # v[t] = cos(omega t) (exact in bf16 for omega = pi/2, pi), x3 = 1: once the
+    # transients p^t have died out, conv[t] = Re(H(e^{j omega}) e^{j omega t})
+    # with the transfer function H(z) = sum_n R_n / (1 - p_n z^-1).
+    L, D, N = 600, 3, 4
+    g = np.random.default_rng(8)
+    a = np.log(g.uniform(0.05, 0.9, (D, N))).astype(np.float32)     # |p| <= 0.9: p^300 < 1e-13
+    R = g.standard_normal((D, N)).astype(np.float32)
+    t = np.arange(L)
+    x1 = np.round(np.cos(omega * t)).astype(np.float32)[None, :, None].repeat(D, 2)  # exactly 1, 0, -1
+    y, _ = oracle.modal_recurrence(bits(x1), ones_bits((1, L, D)), ones_bits((1, L, D)), a, R)
+    for c in range(D):
+        p = np.exp(a[c].astype(np.float64))
+        H = np.sum(R[c].astype(np.float64) / (1.0 - p * np.exp(-1j * omega)))
+        ref = np.real(H * np.exp(1j * omega * t))
+        np.testing.assert_allclose(y[0, 300:, c], ref[300:], rtol=1e-10, atol=1e-10)
+
+
 def test_skip_sits_outside_the_gate():
     # R = 0: y = Dskip * v, whatever x3 is (reading: the skip is not gated by x3).
     inp, S = small_modal()

@@ -268,6 +268,36 @@ def oracle_threads():
         return os.cpu_count() or 1
 
 
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
+def oracle_single_thread_rate(workload, target_s=2.0):
+    """The oracle's rate on one host thread (OpenMP fixed to 1 thread in a child
+    process, since the thread count is read when the oracle library loads)."""
+    import subprocess
+    code = ("import bench, json, os; os.environ['OMP_NUM_THREADS'] = '1'; "
+            f"r, smp, th = bench.oracle_sample_rate(bench.WORKLOADS[{workload!r}], {target_s!r}); "
+            "print(json.dumps([r, smp, th]))")
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    try:
+        out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True,
+                             timeout=120, check=True).stdout.strip().splitlines()[-1]
+        rate, sample, _ = json.loads(out)
+        return rate, sample
+    except Exception as e:  # a baseline detail: report why it is missing instead of failing the bench
+        return None, f"not measured: {type(e).__name__}"
+
+
 def oracle_sample_rate(wl, target_s=10.0):
     """Times the fp64 oracle (as it stands) on a bounded sample of the workload.
 
@@ -615,8 +645,10 @@ def run_gpu(args, wl):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, sample, threads = oracle_sample_rate(wl, args.cpu_seconds)
+        rate1, sample1 = oracle_single_thread_rate(args.workload)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
-                                "sample": sample}
+                                "sample": sample, "cpu_model": cpu_model(),
+                                "single_thread": {"value": rate1, "sample": sample1}}
     if pg is not None:
         pg.barrier()
         pg.destroy_process_group()

@@ -81,7 +81,8 @@ int hyena_oracle_modal_recurrence(int B, int L, int D, int N,
                                   const float *Dskip, const double *state_in,
                                   double *y, double *state_out)
 {
-    if (check_common(B, L, D, ld_x, x1, x2, x3, y) || N < 1 || !log_poles ||
+    /* The per-channel mode arrays below hold at most 256 modes. */
+    if (check_common(B, L, D, ld_x, x1, x2, x3, y) || N < 1 || N > 256 || !log_poles ||
         !residues)
         return ORACLE_BAD_ARG;
     const long long BD = (long long)B * D;
@@ -89,7 +90,6 @@ int hyena_oracle_modal_recurrence(int B, int L, int D, int N,
     for (long long bc = 0; bc < BD; ++bc) {
         const int b = (int)(bc / D), c = (int)(bc % D);
         double p[256], R[256], s[256];
-        if (N > 256) continue;
         for (int n = 0; n < N; ++n) {
             p[n] = exp((double)log_poles[(size_t)c * N + n]);
             R[n] = (double)residues[(size_t)c * N + n];
@@ -340,7 +340,9 @@ int hyena_oracle_fir(int B, int L, int D, int K,
                      int64_t ld_x, const uint16_t *taps, const float *Dskip,
                      const double *hist_in, double *y, double *hist_out)
 {
-    if (check_common(B, L, D, ld_x, x1, x2, x3, y) || K < 1 || !taps)
+    /* The history gather below holds at most 128 values (K <= 129). */
+    if (check_common(B, L, D, ld_x, x1, x2, x3, y) || K < 1 || !taps ||
+        (hist_out && K - 1 > 128))
         return ORACLE_BAD_ARG;
     const long long BD = (long long)B * D;
     const int H = K - 1;
@@ -366,7 +368,6 @@ int hyena_oracle_fir(int B, int L, int D, int K,
         if (hist_out && H > 0) {
             /* Gather first, then write, so hist_out may alias hist_in. */
             double tmp[128];
-            if (H > 128) continue;
             for (int j = 0; j < H; ++j) tmp[j] = V_AT(L - H + j);
             for (int j = 0; j < H; ++j) hist_out[((size_t)b * H + j) * D + c] = tmp[j];
         }

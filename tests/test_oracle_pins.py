@@ -415,3 +415,20 @@ def test_inputs_are_deterministic_and_bf16():
     # rounding is to nearest even: 1 + 2^-8 (a tie) rounds down to 1
     assert f32_to_bf16_bits(np.array([1 + 2 ** -8], np.float32))[0] == 0x3F80
     assert f32_to_bf16_bits(np.array([1 + 3 * 2 ** -8], np.float32))[0] == 0x3F82
+
+
+def test_oracle_refuses_sizes_it_cannot_hold():
+    # The oracle keeps at most 256 modes and a 128-value FIR history per
+    # channel; beyond that it must refuse the call, never leave outputs unwritten.
+    x = np.zeros((1, 4, 8), np.uint16)
+    a = np.full((8, 257), -0.5, np.float32)
+    with pytest.raises(ValueError):
+        oracle.modal_recurrence(x, x, x, a, np.ones_like(a))
+    taps = np.zeros((8, 130), np.uint16)
+    with pytest.raises(ValueError):
+        oracle.fir(x, x, x, taps)
+    # the largest supported sizes still run and fill every output
+    y, S = oracle.modal_recurrence(x, x, x, a[:, :256], np.ones_like(a[:, :256]))
+    assert np.all(np.isfinite(y)) and np.all(S == 0.0)
+    y, H = oracle.fir(x, x, x, taps[:, :129])
+    assert np.all(y == 0.0) and H.shape == (1, 128, 8) and np.all(H == 0.0)

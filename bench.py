@@ -483,6 +483,12 @@ class Step:
         else:
             self._run()
 
+    def check(self):
+        """Raises if a bounded wait inside a modal launch gave up (the timed
+        launches would then have produced wrong results quickly)."""
+        if getattr(self, "ws", None) is not None:
+            self.hy.workspace_check(self.ws)
+
 
 def time_steps(step, steps, warmup, device):
     import torch
@@ -552,6 +558,8 @@ def e2e_leg(wl, host, dev, device, steps, warmup):
         y_host.copy_(y.view(torch.int16), non_blocking=True)
 
     per = time_steps(step, steps, warmup, device)
+    if wl["kind"] == "modal":
+        hy.workspace_check(ws)  # a launch whose bounded wait gave up is an error, not a timing
     h2d = sum(v.numel() * v.element_size() for v in hx.values())
     d2h = y_host.numel() * y_host.element_size()
     return per, h2d, d2h
@@ -588,6 +596,7 @@ def run_gpu(args, wl):
         clk.mark("start")
         per = time_steps(step, args.steps, 0, device)
         clk.mark("end")
+    step.check()
     barrier()
     t_total_ms = max_over_ranks(pg, [sum(per)], device)[0]
     ms_step = t_total_ms / args.steps

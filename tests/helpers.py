@@ -75,3 +75,71 @@ def assert_close(y, ref, what="y", per_channel=False):
         assert worst <= MAX_ABS_TOL, f"{what}: per-channel max-abs {worst:.3e} > {MAX_ABS_TOL}"
         return rel, worst
     return rel, mabs
+
+
+class StreamedCompare:
+    """The acceptance metrics of ``metrics`` / ``assert_close`` over a whole
+    output tensor that is compared block of channels by block of channels
+    (the oracle of a long workload does not fit in host memory at once).
+
+    Feed it (y block, reference block, first channel) pairs covering every
+    channel once; ``result()`` gives (rel-L2, max-abs beyond the bf16
+    rounding / rms(ref)) over the whole tensor and, per channel, the worst
+    max-abs against that channel's own rms and its rel-L2.
+    """
+
+    def __init__(self, D):
+        self.D = D
+        self.sq_err = 0.0
+        self.sq_ref = 0.0
+        self.count = 0
+        self.max_excess = 0.0
+        self.ch_excess = np.zeros(D)
+        self.ch_sq_ref = np.zeros(D)
+        self.ch_sq_err = np.zeros(D)
+        self.ch_count = np.zeros(D)
+        self.seen = np.zeros(D, dtype=bool)
+        self.finite = True
+
+    def add(self, y, ref, c0):
+        y = np.asarray(y, dtype=np.float64)
+        ref = np.asarray(ref, dtype=np.float64)
+        assert y.shape == ref.shape, (y.shape, ref.shape)
+        cb = y.shape[-1]
+        assert not self.seen[c0:c0 + cb].any(), "channel compared twice"
+        self.seen[c0:c0 + cb] = True
+        self.finite &= bool(np.all(np.isfinite(y)))
+        d = np.abs(y - ref).reshape(-1, cb)
+        r = ref.reshape(-1, cb)
+        excess = np.maximum(d - ROUNDING_ALLOWANCE * np.abs(r), 0.0)
+        self.sq_err += float(np.sum(d * d))
+        self.sq_ref += float(np.sum(r * r))
+        self.count += r.size
+        self.max_excess = max(self.max_excess, float(excess.max()) if excess.size else 0.0)
+        self.ch_excess[c0:c0 + cb] = np.max(excess, axis=0)
+        self.ch_sq_ref[c0:c0 + cb] = np.sum(r * r, axis=0)
+        self.ch_sq_err[c0:c0 + cb] = np.sum(d * d, axis=0)
+        self.ch_count[c0:c0 + cb] = r.shape[0]
+
+    def result(self):
+        assert self.seen.all(), "some channels were never compared"
+        rel = float(np.sqrt(self.sq_err / max(self.sq_ref, 1e-300)))
+        rms = float(np.sqrt(self.sq_ref / max(self.count, 1)))
+        mabs = self.max_excess / max(rms, 1e-300)
+        rms_c = np.sqrt(self.ch_sq_ref / np.maximum(self.ch_count, 1))
+        ch_mabs = self.ch_excess / np.maximum(rms_c, 1e-300)
+        ch_rel = np.sqrt(self.ch_sq_err / np.maximum(self.ch_sq_ref, 1e-300))
+        return rel, mabs, ch_mabs, ch_rel
+
+    def check(self, what, per_channel=False):
+        assert self.finite, f"{what}: non-finite values"
+        rel, mabs, ch_mabs, ch_rel = self.result()
+        assert rel <= REL_L2_TOL, f"{what}: rel-L2 {rel:.3e} > {REL_L2_TOL}"
+        assert mabs <= MAX_ABS_TOL, f"{what}: max-abs/rms {mabs:.3e} > {MAX_ABS_TOL}"
+        if per_channel:
+            worst = float(ch_mabs.max())
+            assert worst <= MAX_ABS_TOL, f"{what}: per-channel max-abs {worst:.3e} > {MAX_ABS_TOL}"
+        pct = np.percentile(ch_rel, [50, 99, 100])
+        print(f"{what}: rel-L2 {rel:.3e}, max-abs/rms {mabs:.3e}, per-channel max-abs worst "
+              f"{float(ch_mabs.max()):.3e}, per-channel rel-L2 p50/p99/max {pct[0]:.3e}/{pct[1]:.3e}/{pct[2]:.3e}")
+        return rel, mabs

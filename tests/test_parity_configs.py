@@ -1,13 +1,15 @@
 """Parity at the five acceptance workloads' full sizes, in the launch
 configuration the benchmark times.
 
-The 1K- and 32K-token modal workloads (and both FIR workloads, in their own
-files) are compared element by element with the fp64 oracle over the whole
-output tensor.  For the 131K- and 262K-token workloads the
-oracle runs on a sample of channels (every position of those channels), and
-the whole tensor is checked through properties that hold at any size:
-chunked feeding in whole 128-token units reproduces the single pass bit for
-bit, and all outputs are finite.
+Every element of every output tensor is compared with the fp64 oracle: the
+32K-token modal workload in one oracle call, the 131K- and 262K-token
+workloads with the oracle run block of channels by block of channels (its
+fp64 output for the whole tensor would not fit in host memory at once), and
+the FIR workloads in their own file.  Chunked feeding in whole 128-token units
+must also reproduce the single pass bit for bit over the whole tensor, so the
+chunked results are covered by the same comparison.  The 262K-token workload
+(wide per-channel dynamic range) is also held to the max-abs bound channel by
+channel, and its per-channel rel-L2 percentiles are printed.
 """
 import numpy as np
 import pytest
@@ -15,15 +17,11 @@ import pytest
 import oracle
 from synth import WORKLOAD_SHAPES, make_workload_inputs
 
-from .helpers import assert_close, bits_of, from_dev_bf16, metrics, to_dev_bf16, to_dev_f32
+from .helpers import StreamedCompare, assert_close, from_dev_bf16, metrics, to_dev_bf16, to_dev_f32
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
-
-def sample_channels(D, k=40, seed=0):
-    rng = np.random.default_rng(seed)
-    fixed = [0, 1, 62, 63, 64, D // 2, D - 2, D - 1]
-    return np.unique(np.concatenate([fixed, rng.choice(D, size=k, replace=False)]))
+CHANNEL_BLOCK = 256
 
 
 class Dev:
@@ -53,10 +51,23 @@ def modal_run(dev, inp, chunk=None):
     return y, S
 
 
-def sampled_oracle(inp, chans):
-    sub = {k: np.ascontiguousarray(inp[k][:, :, chans]) for k in ("x1", "x2", "x3")}
-    return oracle.modal_recurrence(sub["x1"], sub["x2"], sub["x3"], inp["log_poles"][chans],
-                                   inp["residues"][chans], inp["Dskip"][chans])
+def streamed_oracle_check(y, S, inp, what, per_channel=False):
+    """Every element of y and of the final state against the fp64 recurrence
+    oracle, one block of channels at a time."""
+    D = inp["D"]
+    cmp = StreamedCompare(D)
+    S_host = S.cpu().numpy().astype(np.float64)
+    s_err = s_ref = 0.0
+    for c0 in range(0, D, CHANNEL_BLOCK):
+        c1 = min(D, c0 + CHANNEL_BLOCK)
+        sub = [np.ascontiguousarray(inp[k][:, :, c0:c1]) for k in ("x1", "x2", "x3")]
+        ref_y, ref_S = oracle.modal_recurrence(*sub, inp["log_poles"][c0:c1], inp["residues"][c0:c1],
+                                               inp["Dskip"][c0:c1])
+        cmp.add(from_dev_bf16(y[:, :, c0:c1]), ref_y, c0)
+        s_err += float(np.sum((S_host[:, c0:c1] - ref_S) ** 2))
+        s_ref += float(np.sum(ref_S ** 2))
+    cmp.check(what, per_channel=per_channel)
+    assert np.sqrt(s_err / s_ref) < 1e-4, f"{what}: state rel-L2 {np.sqrt(s_err / s_ref):.3e}"
 
 
 def test_modal_32k_full_tensor():
@@ -79,15 +90,13 @@ def test_modal_131k_chunked_prefill():
     dev = Dev(inp)
     y1, S1 = modal_run(dev, inp)
     yc, Sc = modal_run(dev, inp, chunk=WORKLOAD_SHAPES["modal_131k_chunked"]["chunk"])
-    # 1024-token chunks are whole 128-token units: bitwise equal to the single pass
+    # 1024-token chunks are whole 128-token units: bitwise equal to the single
+    # pass over the whole tensor
     assert torch.equal(yc.view(torch.int16), y1.view(torch.int16))
     assert torch.equal(Sc, S1)
-    chans = sample_channels(inp["D"], seed=3)
-    ref_y, ref_S = sampled_oracle(inp, chans)
-    idx = torch.from_numpy(chans).cuda()
-    assert_close(from_dev_bf16(yc.index_select(2, idx)), ref_y, "modal 131K in 1024-token chunks (sampled channels)")
-    rel, _ = metrics(Sc[:, chans].cpu().numpy().astype(np.float64), ref_S)
-    assert rel < 1e-4
+    del y1
+    torch.cuda.empty_cache()
+    streamed_oracle_check(yc, Sc, inp, "modal 131K in 1024-token chunks")
 
 
 def test_modal_262k_long_context_wide_range():
@@ -95,16 +104,10 @@ def test_modal_262k_long_context_wide_range():
     inp = make_workload_inputs("modal_262k_wide")
     dev = Dev(inp)
     y1, S1 = modal_run(dev, inp)
-    assert bool(torch.isfinite(y1.float()).all())
-    chans = sample_channels(inp["D"], seed=4)
-    ref_y, ref_S = sampled_oracle(inp, chans)
-    idx = torch.from_numpy(chans).cuda()
-    assert_close(from_dev_bf16(y1.index_select(2, idx)), ref_y, "modal 262K single pass", per_channel=True)
-    rel, _ = metrics(S1[:, chans].cpu().numpy().astype(np.float64), ref_S)
-    assert rel < 1e-4
-    y1_bits = bits_of(y1.index_select(2, idx))
-    del y1
-    torch.cuda.empty_cache()
     yc, Sc = modal_run(dev, inp, chunk=1024)
-    assert np.array_equal(bits_of(yc.index_select(2, idx)), y1_bits)
+    # the 1024-chunked feed equals the single pass bit for bit, whole tensor
+    assert torch.equal(yc.view(torch.int16), y1.view(torch.int16))
     assert torch.equal(Sc, S1)
+    del yc
+    torch.cuda.empty_cache()
+    streamed_oracle_check(y1, S1, inp, "modal 262K single pass (and 1024-chunked)", per_channel=True)

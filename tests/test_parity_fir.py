@@ -85,14 +85,9 @@ def test_chunked_is_bitwise_single_pass(K, chunks):
 @pytest.mark.slow
 @pytest.mark.parametrize("K", list(WORKLOAD_SHAPES["fir_8k"]["K"]))
 def test_fir_8k_full_size(K):
-    import torch
+    # every element of the B=2, L=8192, D=4096 output against the oracle
     c = WORKLOAD_SHAPES["fir_8k"]
     inp = make_fir_inputs(c["B"], c["L"], c["D"], K, c["seed"])
     y, _ = run_gpu(inp)
-    rng = np.random.default_rng(K)
-    chans = np.unique(np.concatenate([[0, 1, 63, 64, c["D"] - 1], rng.choice(c["D"], 120, replace=False)]))
-    sub = {k: np.ascontiguousarray(inp[k][:, :, chans]) for k in ("x1", "x2", "x3")}
-    ref, _ = oracle.fir(sub["x1"], sub["x2"], sub["x3"], inp["taps"][chans], None, None)
-    idx = torch.from_numpy(chans).cuda()
-    assert_close(from_dev_bf16(y.index_select(2, idx)), ref, f"FIR 8K K={K}")
-    assert bool(torch.isfinite(y.float()).all())
+    ref, _ = oracle.fir(inp["x1"], inp["x2"], inp["x3"], inp["taps"], None, None)
+    assert_close(from_dev_bf16(y), ref, f"FIR 8K K={K}")

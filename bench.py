@@ -58,6 +58,11 @@ WORKLOADS = {
                          desc="hcs explicit FIR K=7, B=2 L=8192 D=4096, inputs interleaved per channel triple"),
     "fir128_triples": dict(kind="fir", B=2, L=8192, D=4096, K=128, seed=1, group=1,
                            desc="hcm explicit FIR K=128, B=2 L=8192 D=4096, inputs interleaved per channel triple"),
+    # more than 16 real modes (two or four lanes per channel pair)
+    "modal32k_n32": dict(kind="modal", B=1, L=32768, D=4096, N=32, seed=11, chunk=None,
+                         desc="hcl modal long conv, B=1 L=32768 D=4096 N=32, single pass"),
+    "modal32k_n64": dict(kind="modal", B=1, L=32768, D=4096, N=64, seed=12, chunk=None,
+                         desc="hcl modal long conv, B=1 L=32768 D=4096 N=64, single pass"),
     # complex modes, h[t] = Re sum R p^t (the Evo 1 modal form; state size 8)
     "cmodal8k": dict(kind="modal", cx=True, B=1, L=8192, D=4096, N=8, seed=9, chunk=None,
                      desc="complex-mode modal long conv, B=1 L=8192 D=4096 N=8, single pass"),

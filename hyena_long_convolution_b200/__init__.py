@@ -45,8 +45,8 @@ __all__ = [
     "workspace_size",
 ]
 
-MAX_MODES = 16
-MAX_COMPLEX_MODES = 8
+MAX_MODES = 64
+MAX_COMPLEX_MODES = 32
 MAX_TAPS = 128
 
 

@@ -39,6 +39,8 @@ SIGNATURES = {
                                    _I, _I, _I, _I, _P, _SZ, _P]),
     "hyena_modal_long_conv_noalloc": (_I, [_P, _P, _P, _I64, _P, _P, _P, _P, _I64, _P, _P,
                                            _I, _I, _I, _I, _P]),
+    "hyena_modal_noalloc_check": (_I, [_P]),
+    "hyena_modal_noalloc_scratch": (_I, [_P, _P]),
     "hyena_modal_decode": (_I, [_P, _P, _P, _I64, _P, _P, _P, _P, _I64, _P, _I, _I, _I, _P]),
     "hyena_short_decode": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I64, _P, _I, _I, _I, _P]),
     "hyena_short_conv_packed": (_I, [_P, _I64, _I, _P, _P, _P, _I64, _P, _P, _I, _I, _I, _I, _P]),

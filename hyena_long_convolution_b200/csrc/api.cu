@@ -50,10 +50,12 @@ XSource packed_source(const hyena_bf16_t *xp, long long ld, int group)
 }
 
 // 4-D bf16 tensor map [B][L][groups][group] over input k (0..2), box of `rows`
-// tokens x 64 channels: dims {group, D / group, L, B}, the group stride 3 group
-// elements (unused for a single group).  Triples: one map over the interleaved rows, dims {3D, 1, L, B},
-// box of `rows` tokens x 192 values (64 channels' triples).
-bool encode_x_map(CUtensorMap *m, const XSource &xs, int k, int B, int L, int D, int rows)
+// tokens x `width` channels (64, or 32 / 16 for the modal scan's narrower
+// chains): dims {group, D / group, L, B}, the group stride 3 group elements
+// (unused for a single group).  Triples: one map over the interleaved rows,
+// dims {3D, 1, L, B}, box of `rows` tokens x 3 width values (width channels'
+// triples).
+bool encode_x_map(CUtensorMap *m, const XSource &xs, int k, int B, int L, int D, int rows, int width = 64)
 {
     std::call_once(g_encode_once, resolve_encode);
     if (g_encode == nullptr) return false;
@@ -64,19 +66,19 @@ bool encode_x_map(CUtensorMap *m, const XSource &xs, int k, int B, int L, int D,
         dims[0] = 3ull * static_cast<cuuint64_t>(D);
         dims[1] = 1;
         strides[0] = row_bytes;
-        box[0] = 3u * 64u;
+        box[0] = 3u * static_cast<cuuint32_t>(width);
         box[1] = 1u;
     } else {
         const int groups = D / xs.group;
         dims[0] = static_cast<cuuint64_t>(xs.group);
         dims[1] = static_cast<cuuint64_t>(groups);
         strides[0] = groups > 1 ? 6ull * static_cast<cuuint64_t>(xs.group) : row_bytes;
-        // 64 channels per box: one run of 64 within a group (a single group
-        // reads past its end as zeros), or 64 / group whole groups of fewer
-        // than 64 channels (group divides 64)
-        const bool runs = groups == 1 || xs.group >= 64;
-        box[0] = static_cast<cuuint32_t>(runs ? 64 : xs.group);
-        box[1] = static_cast<cuuint32_t>(runs ? 1 : 64 / xs.group);
+        // `width` channels per box: one run of width within a group (a single
+        // group reads past its end as zeros), or width / group whole groups of
+        // fewer channels (group divides width)
+        const bool runs = groups == 1 || xs.group >= width;
+        box[0] = static_cast<cuuint32_t>(runs ? width : xs.group);
+        box[1] = static_cast<cuuint32_t>(runs ? 1 : width / xs.group);
     }
     dims[2] = static_cast<cuuint64_t>(L);
     dims[3] = static_cast<cuuint64_t>(B);
@@ -150,12 +152,16 @@ void record_cuda_error(cudaError_t e, const char *where)
 
 void record_message(const char *msg) { snprintf(g_last_error, sizeof g_last_error, "%s", msg); }
 
+void add_launches(int n) { g_last_launches += n; }
+
 ModalLayout modal_layout(int B, int D, int N)
 {
     ModalLayout L;
     L.NP = modal_padded_modes(N);
-    L.nCB = (D + MCH - 1) / MCH;
-    L.Dp = L.nCB * MCH;
+    L.LPC = modal_lanes_per_pair(L.NP);
+    const int width = MCH / L.LPC;  // channels per chain
+    L.nCB = (D + width - 1) / width;
+    L.Dp = L.nCB * width;
     const size_t row = static_cast<size_t>(L.Dp) * sizeof(float);
     size_t off = 0;
     L.off_hdr = off;
@@ -166,7 +172,7 @@ ModalLayout modal_layout(int B, int D, int N)
     L.off_flags = off;
     off = align256(off + chains * MRING * sizeof(unsigned long long));
     L.off_slots = off;
-    off = align256(off + chains * MRING * (MGMAX + 1) * L.NP * MCH * sizeof(float));
+    off = align256(off + chains * MRING * (MGMAX + 1) * L.NP * width * sizeof(float));
     L.total = off;
     return L;
 }
@@ -296,13 +302,20 @@ hyena_status_t modal_long_conv_impl(const XSource &xs, const float *log_poles, c
     sy.Dp = lay.Dp;
     sy.coef = reinterpret_cast<float *>(ws + lay.off_coef);
 
-    CUtensorMap m1, m2, m3;
-    if (!encode_x_map(&m1, xs, 0, B, L, D, MCK)) return HYENA_ERR_CUDA;
-    if (xs.triples)
-        m2 = m3 = m1;
-    else if (!encode_x_map(&m2, xs, 1, B, L, D, MCK) || !encode_x_map(&m3, xs, 2, B, L, D, MCK))
+    ModalMaps maps;
+    const int width = MCH / lay.LPC;  // channels per chain
+    if (!encode_x_map(&maps.a1, xs, 0, B, L, D, MA_ROWS, width) ||
+        !encode_x_map(&maps.c1, xs, 0, B, L, D, MC_ROWS, width))
         return HYENA_ERR_CUDA;
-    const int n = launch_modal(m1, m2, m3, a, sy, lay.NP, xs.triples, cx, s);
+    if (xs.triples) {
+        maps.a2 = maps.a1;
+        maps.c2 = maps.c3 = maps.c1;
+    } else if (!encode_x_map(&maps.a2, xs, 1, B, L, D, MA_ROWS, width) ||
+               !encode_x_map(&maps.c2, xs, 1, B, L, D, MC_ROWS, width) ||
+               !encode_x_map(&maps.c3, xs, 2, B, L, D, MC_ROWS, width)) {
+        return HYENA_ERR_CUDA;
+    }
+    const int n = launch_modal(maps, a, sy, lay.NP, xs.triples, cx, s);
     if (n < 0) return HYENA_ERR_CUDA;
     g_last_launches = n;
     return HYENA_OK;

@@ -34,14 +34,16 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits(float f)
 
 constexpr int kDecodeThreads = 64;  // small blocks: more CTAs (SMs) per call at batch 1
 
-// N consecutive floats at p (16-byte aligned when N % 4 == 0) into v[0, N).
-template <int NP>
-__device__ __forceinline__ void load_row(float (&v)[NP], const float *p, int N)
+// The NB floats p[i] for slots i of [base, base + NB) that exist (i < N) into
+// v[0, NB), zero beyond N; 16-byte loads when the whole block exists and is
+// aligned (N a multiple of 4).
+template <int NB>
+__device__ __forceinline__ void load_block(float (&v)[NB], const float *p, int base, int N)
 {
-    if (N == NP) {
+    if (base + NB <= N && (N & 3) == 0) {
 #pragma unroll
-        for (int i = 0; i < NP; i += 4) {
-            const float4 q = __ldg(reinterpret_cast<const float4 *>(p + i));
+        for (int i = 0; i < NB; i += 4) {
+            const float4 q = __ldg(reinterpret_cast<const float4 *>(p + base + i));
             v[i] = q.x;
             v[i + 1] = q.y;
             v[i + 2] = q.z;
@@ -49,16 +51,22 @@ __device__ __forceinline__ void load_row(float (&v)[NP], const float *p, int N)
         }
     } else {
 #pragma unroll
-        for (int i = 0; i < NP; ++i) v[i] = i < N ? p[i] : 0.f;
+        for (int i = 0; i < NB; ++i) v[i] = base + i < N ? p[base + i] : 0.f;
     }
 }
 
 // kCx: complex modes, N counts slots (two per mode, as the prefill kernel's
 // coefficient table): the pole pair is used as given and the residue pair as
 // (Re R, -Im R); the state update is the prefill kernel's complex step.
-template <int NP, bool kCx>
+// NPT padded slots are taken in blocks of NB = min(NPT, 16), the slots one
+// lane of the prefill kernel holds: each block's part of the readout is formed
+// with the same two accumulation chains, and the parts are added in the
+// prefill kernel's butterfly order ((p0 + p1) + (p2 + p3)).
+template <int NPT, bool kCx>
 __global__ void __launch_bounds__(kDecodeThreads) modal_decode_kernel(const DecodeArgs A)
 {
+    constexpr int NB = NPT < 16 ? NPT : 16;
+    constexpr int NBLK = NPT / NB;
     const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (idx >= static_cast<long long>(A.B) * A.D) return;
     const int b = static_cast<int>(idx / A.D);
@@ -67,56 +75,69 @@ __global__ void __launch_bounds__(kDecodeThreads) modal_decode_kernel(const Deco
     const float v = __fmul_rn(bf16_bits_to_float(A.x1[xi]), bf16_bits_to_float(A.x2[xi]));
     const float x3 = bf16_bits_to_float(A.x3[xi]);
     float *st = A.state + (static_cast<size_t>(b) * A.D + c) * A.N;
+    const float *ap = A.log_poles + static_cast<size_t>(c) * A.N;
+    const float *rp = A.residues + static_cast<size_t>(c) * A.N;
 
-    // padded modes (n >= N): p = R = 0 and a zero state, as in the prefill kernel
-    float a[NP], r[NP], s[NP];
-    load_row<NP>(a, A.log_poles + static_cast<size_t>(c) * A.N, A.N);
-    load_row<NP>(r, A.residues + static_cast<size_t>(c) * A.N, A.N);
-    if (A.N == NP) {
+    float part[NBLK];
 #pragma unroll
-        for (int i = 0; i < NP; i += 4) {
-            const float4 q = *reinterpret_cast<const float4 *>(st + i);
-            s[i] = q.x;
-            s[i + 1] = q.y;
-            s[i + 2] = q.z;
-            s[i + 3] = q.w;
+    for (int bi = 0; bi < NBLK; ++bi) {
+        const int base = bi * NB;
+        // padded slots (>= N): p = R = 0 and a zero state, as in the prefill kernel
+        float a[NB], r[NB], s[NB];
+        load_block<NB>(a, ap, base, A.N);
+        load_block<NB>(r, rp, base, A.N);
+        if (base + NB <= A.N && (A.N & 3) == 0) {
+#pragma unroll
+            for (int i = 0; i < NB; i += 4) {
+                const float4 q = *reinterpret_cast<const float4 *>(st + base + i);
+                s[i] = q.x;
+                s[i + 1] = q.y;
+                s[i + 2] = q.z;
+                s[i + 3] = q.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < NB; ++i) s[i] = base + i < A.N ? st[base + i] : 0.f;
         }
-    } else {
+        if constexpr (!kCx) {
 #pragma unroll
-        for (int i = 0; i < NP; ++i) s[i] = i < A.N ? st[i] : 0.f;
-    }
-    if constexpr (!kCx) {
+            for (int n = 0; n < NB; ++n) s[n] = __fmaf_rn(base + n < A.N ? expf(a[n]) : 0.f, s[n], v);
+        } else {
+            // a[] holds the poles (zero in padded slots); residue pairs (Re, -Im)
 #pragma unroll
-        for (int n = 0; n < NP; ++n) s[n] = __fmaf_rn(n < A.N ? expf(a[n]) : 0.f, s[n], v);
-    } else {
-        // a[] holds the poles (zero in padded slots); residue pairs (Re, -Im)
+            for (int m = 0; m < NB; m += 2) {
+                r[m + 1] = -r[m + 1];
+                const float re = s[m], im = s[m + 1];
+                s[m] = __fmaf_rn(a[m], re, __fmaf_rn(-a[m + 1], im, v));
+                s[m + 1] = __fmaf_rn(a[m], im, __fmul_rn(a[m + 1], re));
+            }
+        }
+        float a0 = __fmul_rn(r[0], s[0]);
+        float a1 = __fmul_rn(r[1], s[1]);
 #pragma unroll
-        for (int m = 0; m < NP; m += 2) {
-            r[m + 1] = -r[m + 1];
-            const float re = s[m], im = s[m + 1];
-            s[m] = __fmaf_rn(a[m], re, __fmaf_rn(-a[m + 1], im, v));
-            s[m + 1] = __fmaf_rn(a[m], im, __fmul_rn(a[m + 1], re));
+        for (int n = 2; n < NB; n += 2) {
+            a0 = __fmaf_rn(r[n], s[n], a0);
+            a1 = __fmaf_rn(r[n + 1], s[n + 1], a1);
+        }
+        part[bi] = __fadd_rn(a0, a1);
+        if (base + NB <= A.N && (A.N & 3) == 0) {
+#pragma unroll
+            for (int i = 0; i < NB; i += 4)
+                *reinterpret_cast<float4 *>(st + base + i) = make_float4(s[i], s[i + 1], s[i + 2], s[i + 3]);
+        } else {
+#pragma unroll
+            for (int n = 0; n < NB; ++n)
+                if (base + n < A.N) st[base + n] = s[n];
         }
     }
-    float a0 = __fmul_rn(r[0], s[0]);
-    float a1 = __fmul_rn(r[1], s[1]);
+    // butterfly: neighbours first, then pairs of neighbours
 #pragma unroll
-    for (int n = 2; n < NP; n += 2) {
-        a0 = __fmaf_rn(r[n], s[n], a0);
-        a1 = __fmaf_rn(r[n + 1], s[n + 1], a1);
-    }
-    const float conv = __fadd_rn(a0, a1);
+    for (int d = 1; d < NBLK; d <<= 1)
+#pragma unroll
+        for (int bi = 0; bi < NBLK; bi += 2 * d) part[bi] = __fadd_rn(part[bi], part[bi + d]);
+    const float conv = part[0];
     const float dsk = A.Dskip != nullptr ? A.Dskip[c] : 0.f;
     A.y[static_cast<size_t>(b) * A.ld_y + c] = float_to_bf16_bits(__fmaf_rn(dsk, v, __fmul_rn(x3, conv)));
-    if (A.N == NP) {
-#pragma unroll
-        for (int i = 0; i < NP; i += 4)
-            *reinterpret_cast<float4 *>(st + i) = make_float4(s[i], s[i + 1], s[i + 2], s[i + 3]);
-    } else {
-#pragma unroll
-        for (int n = 0; n < NP; ++n)
-            if (n < A.N) st[n] = s[n];
-    }
 }
 
 // hist [B, K-1, D] in time order: hist[b][K-2][c] is v of the previous token.
@@ -175,14 +196,23 @@ int launch_modal_decode(const DecodeArgs &a, bool cx, cudaStream_t st)
 {
     const long long n = static_cast<long long>(a.B) * a.D;
     const unsigned int grid = static_cast<unsigned int>((n + kDecodeThreads - 1) / kDecodeThreads);
-    switch (modal_padded_modes(a.N) + (cx ? 1 : 0)) {
-        case 4: modal_decode_kernel<4, false><<<grid, kDecodeThreads, 0, st>>>(a); break;
-        case 8: modal_decode_kernel<8, false><<<grid, kDecodeThreads, 0, st>>>(a); break;
-        case 16: modal_decode_kernel<16, false><<<grid, kDecodeThreads, 0, st>>>(a); break;
-        case 5: modal_decode_kernel<4, true><<<grid, kDecodeThreads, 0, st>>>(a); break;
-        case 9: modal_decode_kernel<8, true><<<grid, kDecodeThreads, 0, st>>>(a); break;
-        default: modal_decode_kernel<16, true><<<grid, kDecodeThreads, 0, st>>>(a); break;
+    const int npt = modal_padded_modes(a.N);
+#define HYENA_DECODE_CASE(NPT)                                                                  \
+    case NPT:                                                                                    \
+        if (cx)                                                                                  \
+            modal_decode_kernel<NPT, true><<<grid, kDecodeThreads, 0, st>>>(a);                  \
+        else                                                                                     \
+            modal_decode_kernel<NPT, false><<<grid, kDecodeThreads, 0, st>>>(a);                 \
+        break;
+    switch (npt) {
+        HYENA_DECODE_CASE(4)
+        HYENA_DECODE_CASE(8)
+        HYENA_DECODE_CASE(16)
+        HYENA_DECODE_CASE(32)
+        HYENA_DECODE_CASE(64)
+        default: return -1;
     }
+#undef HYENA_DECODE_CASE
     HYENA_TRY(cudaGetLastError(), "modal decode launch");
     return 1;
 }

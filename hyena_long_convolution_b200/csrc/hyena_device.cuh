@@ -15,6 +15,7 @@ enum : unsigned int {
     kErrLookbackTimeout = 1u,
     kErrTmaTimeout = 2u,
     kErrRingTimeout = 4u,
+    kErrLocalTimeout = 8u,  // a hand-off between a CTA's own warps ran out
 };
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
@@ -58,6 +59,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking test: true if the phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(smem_u32(bar)), "r"(parity)
@@ -195,22 +210,29 @@ __device__ __forceinline__ void modes_step(float2 (&s)[NP], const float2 (&p)[NP
     }
 }
 
-// One carry step, C <- P C + A with a full state A (P = p^MT).
+// One carry step of a slot pair (two real modes, or the real and imaginary
+// slots of one complex mode), C <- P C + A with a full state A (P = p^k).
+template <bool kCx>
+__device__ __forceinline__ void carry_pair(float2 &c0, float2 &c1, float2 P0, float2 P1, float2 A0, float2 A1)
+{
+    if constexpr (!kCx) {
+        c0 = __ffma2_rn(P0, c0, A0);
+        c1 = __ffma2_rn(P1, c1, A1);
+    } else {
+        const float2 re = c0, im = c1;
+        const float2 npi = make_float2(-P1.x, -P1.y);
+        c0 = __ffma2_rn(P0, re, __ffma2_rn(npi, im, A0));
+        c1 = __ffma2_rn(P0, im, __ffma2_rn(P1, re, A1));
+    }
+}
+
+// One carry step of all NP slots, C <- P C + A (the same operations as
+// carry_pair on each slot pair).
 template <int NP, bool kCx>
 __device__ __forceinline__ void modes_carry(float2 (&C)[NP], const float2 (&P)[NP], const float2 (&A)[NP])
 {
-    if constexpr (!kCx) {
 #pragma unroll
-        for (int n = 0; n < NP; ++n) C[n] = __ffma2_rn(P[n], C[n], A[n]);
-    } else {
-#pragma unroll
-        for (int m = 0; m < NP; m += 2) {
-            const float2 re = C[m], im = C[m + 1];
-            const float2 npi = make_float2(-P[m + 1].x, -P[m + 1].y);
-            C[m] = __ffma2_rn(P[m], re, __ffma2_rn(npi, im, A[m]));
-            C[m + 1] = __ffma2_rn(P[m], im, __ffma2_rn(P[m + 1], re, A[m + 1]));
-        }
-    }
+    for (int m = 0; m < NP; m += 2) carry_pair<kCx>(C[m], C[m + 1], P[m], P[m + 1], A[m], A[m + 1]);
 }
 
 __device__ __forceinline__ float2 ldg_f2(const float *p)

@@ -15,6 +15,9 @@ namespace hyena {
 // hyena_last_error_message).
 void record_cuda_error(cudaError_t e, const char *where);
 void record_message(const char *msg);
+// Adds to the launch count that hyena_last_launch_count reports for the
+// calling thread's most recent call.
+void add_launches(int n);
 
 #define HYENA_TRY(call, where)                       \
     do {                                             \
@@ -41,25 +44,40 @@ __host__ __device__ __forceinline__ long long x_col(int c, int group)
 
 // ---------------------------------------------------------------- modal scan
 // A chain is the sequence of MCH channels of one batch row over time.  A unit
-// is MT consecutive tokens of a chain, swept by one warp (lane l owns the
-// channel pair 2l, 2l+1); a group is G consecutive units handled by one CTA of
-// G compute warps plus a control warp.  Tiles stream through shared memory in
-// chunks of MCK rows.
+// is MT consecutive tokens of a chain: the carry from one unit to the next
+// follows one canonical fp32 recurrence, so feeding a sequence in chunks of
+// whole units reproduces the single pass bit for bit.  A group is MGMAX
+// consecutive units of a chain, the work item one CTA takes at a time: one
+// aggregate warp per unit and one output warp per half unit (MH tokens).
+// Up to 16 mode slots per lane: lane l of a warp owns the channel pair 2l,
+// 2l+1 of a 64-channel chain and all its (padded) mode slots.  With 32 or 64
+// slots, LPC = 2 or 4 lanes share a channel pair, each owning 16 consecutive
+// slots, and a chain is 64 / LPC channels wide.
 constexpr int MCH = 64;
 constexpr int MT = 128;
-constexpr int MCK = 16;
+constexpr int MH = MT / 2;
 constexpr int MRING = 16;  // group slots per chain
 constexpr int MLB = 8;     // deepest look-back, in groups
-constexpr int MGMAX = 4;   // largest group (slots are sized for it)
+constexpr int MGMAX = 4;   // units per group (slots are sized for it)
 
-inline int modal_padded_modes(int N) { return N <= 4 ? 4 : (N <= 8 ? 8 : 16); }
+constexpr int MSLOTS_LANE = 16;  // most mode slots one lane holds
 
-// Coefficient table [3NP+1][Dp]: rows [0, NP) p = exp(a), [NP, 2NP) residues,
-// row 2NP Dskip, rows [2NP+1, 3NP+1) p^MT.
-inline int modal_coef_rows(int NP) { return 3 * NP + 1; }
+// Padded mode slots per channel (NPT): 4, 8, 16, 32 or 64.
+inline int modal_padded_modes(int N) { return N <= 4 ? 4 : (N <= 8 ? 8 : (N <= 16 ? 16 : (N <= 32 ? 32 : 64))); }
+// Lanes per channel pair (LPC) and slots per lane for NPT padded slots.
+inline int modal_lanes_per_pair(int NPT) { return NPT <= MSLOTS_LANE ? 1 : NPT / MSLOTS_LANE; }
+inline int modal_lane_slots(int NPT) { return NPT <= MSLOTS_LANE ? NPT : MSLOTS_LANE; }
+
+// Coefficient table [4NPT+1][Dp]: rows [0, NPT) p = exp(a), [NPT, 2NPT)
+// residues, row 2NPT Dskip, rows [2NPT+1, 3NPT+1) p^MT, rows [3NPT+1, 4NPT+1)
+// p^MH.
+inline int modal_coef_rows(int NPT) { return 4 * NPT + 1; }
 
 struct ModalLayout {
-    int NP = 0, nCB = 0, Dp = 0;
+    int NP = 0;    // padded mode slots per channel (NPT)
+    int LPC = 1;   // lanes per channel pair
+    int nCB = 0;   // chains per batch row (chain width MCH / LPC)
+    int Dp = 0;
     size_t off_hdr = 0, off_coef = 0, off_flags = 0, off_slots = 0, total = 0;
 };
 
@@ -74,12 +92,12 @@ struct ModalArgs {
     const float *state_in;
     float *state_out;
     int B, L, D, N;
-    int nCB, Dp;
+    int nCB, Dp;                // chains per batch row (MCH / LPC channels each), nCB * chain width
     int units;                  // units per chain, ceil(L / MT)
     unsigned int nGroups;       // groups over all chains
-    const float *coef;          // [3NP+1][Dp]
+    const float *coef;          // [4NPT+1][Dp]
     unsigned long long *flags;  // [B*nCB][MRING]
-    float *slots;               // [B*nCB][MRING][MGMAX+1][NP][MCH]
+    float *slots;               // [B*nCB][MRING][MGMAX+1][NPT][chain width]
     unsigned int *hdr;          // [0] ticket, [1] finished CTAs, [2] error bits, [3] epoch
 };
 
@@ -92,15 +110,24 @@ struct ModalSynthArgs {
     float *coef;
 };
 
+// Rows of the tensor-map boxes the scan kernel reads: aggregate warps take
+// MA_ROWS tokens per chunk (x1, x2), output warps MC_ROWS (x1, x2, x3).
+constexpr int MA_ROWS = 16;
+constexpr int MC_ROWS = 8;
+
 // Launches the coefficient-synthesis kernel and the scan kernel; returns the
-// number of launches enqueued or a negative value on a CUDA error.  The three
-// 4-D tensor maps [B][L][groups][group] cover x1, x2, x3 with boxes of MCK rows
-// x MCH channels; with `triples` the first map alone covers the interleaved
-// rows (box MCK rows x 3 MCH elements) and the other two are unused.
-// With `cx` the N of the arguments counts mode slots, two per complex mode
-// (state [B][D][N/2][2] = [B][D][N]).
-int launch_modal(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3,
-                 ModalArgs a, const ModalSynthArgs &s, int NP, bool triples, bool cx, cudaStream_t st);
+// number of launches enqueued or a negative value on a CUDA error.  The 4-D
+// tensor maps [B][L][groups][group] cover x1, x2 (a1, a2: boxes of MA_ROWS
+// rows x MCH channels) and x1, x2, x3 (c1..c3: boxes of MC_ROWS rows); with
+// `triples` a1 and c1 alone cover the interleaved rows (boxes of 3 MCH
+// elements per row) and the others are unused.  With `cx` the N of the
+// arguments counts mode slots, two per complex mode (state [B][D][N/2][2] =
+// [B][D][N]).
+struct ModalMaps {
+    CUtensorMap a1, a2, c1, c2, c3;
+};
+int launch_modal(const ModalMaps &maps, ModalArgs a, const ModalSynthArgs &s, int NPT, bool triples, bool cx,
+                 cudaStream_t st);
 
 // ---------------------------------------------------------------- short FIR
 constexpr int FCH = 64;   // channels per CTA

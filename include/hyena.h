@@ -69,8 +69,8 @@ const char *hyena_status_string(hyena_status_t s);
 int hyena_abi_version(void);
 
 /* Largest supported number of modes N (real; complex) and of FIR taps K. */
-#define HYENA_MAX_MODES 16
-#define HYENA_MAX_COMPLEX_MODES 8
+#define HYENA_MAX_MODES 64
+#define HYENA_MAX_COMPLEX_MODES 32
 #define HYENA_MAX_TAPS 128
 
 /*
@@ -164,9 +164,13 @@ hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t 
  * device, with that device current); make that first call before any stream
  * capture.  All calls share the one array: calls that overlap on the GPU (on
  * different streams, or from different threads without ordering) race and
- * produce wrong results.  Each call clears the array's counters before its
- * launch; a bounded-wait timeout inside the kernel invalidates that call's
- * output and is not reported by this entry point.
+ * produce wrong results.  Before its scan, each call enqueues one small
+ * kernel that moves the previous call's device-side error bits aside and
+ * zeroes the look-back flags of its own (B, D, N) layout.  A bounded device
+ * wait that runs out invalidates that call's output; the call itself returns
+ * before the GPU runs, so it cannot report it: hyena_modal_noalloc_check does.
+ * The cached device address is valid for the device's current context only:
+ * do not use this entry point across a device reset.
  */
 #define HYENA_NOALLOC_SCRATCH_BYTES (24u << 20)
 
@@ -177,6 +181,29 @@ hyena_status_t hyena_modal_long_conv_noalloc(const hyena_bf16_t *x1, const hyena
                                              hyena_bf16_t *y, int64_t ld_y,
                                              const float *state_in, float *state_out,
                                              int B, int L, int D, int N, void *stream);
+
+/*
+ * Reports device-side failures of hyena_modal_long_conv_noalloc calls on the
+ * current device (no counterpart on the pages; the allocation-free
+ * counterpart of hyena_workspace_check).  Synchronises `stream`, then returns
+ * HYENA_ERR_TIMEOUT if a bounded wait ran out in any call since the previous
+ * check (that call's y and state_out are invalid; later calls are not
+ * affected) and clears the record; HYENA_OK otherwise.  Allocates nothing.
+ */
+hyena_status_t hyena_modal_noalloc_check(void *stream);
+
+/*
+ * The device address and size of the fixed scratch array that
+ * hyena_modal_long_conv_noalloc uses on the current device (no counterpart on
+ * the pages), for callers that account for device memory or that want to
+ * inspect it.  The array's header holds, as 32-bit words: [0] the next group
+ * ticket, [1] finished CTAs, [2] error bits of the running call, [3] the
+ * launch epoch, [4] error bits not yet reported by hyena_modal_noalloc_check.
+ * Writing to the array while a call runs corrupts that call.  The first use
+ * on a device performs the address look-up (make it before any stream
+ * capture).
+ */
+hyena_status_t hyena_modal_noalloc_scratch(void **device_ptr, size_t *bytes);
 
 /*
  * One generated token through the long modal filter: the recurrent form of
@@ -331,7 +358,13 @@ hyena_status_t hyena_modal_decode_complex_packed(const hyena_bf16_t *xp, int64_t
 
 /*
  * Zero-fills a modal state [B, D, N] fp32 (the state before the first token
- * of a sequence): the start of chunked prefill.
+ * of a sequence): the start of chunked prefill.  The carried IIR state is the
+ * cache that the Evo2-7B-262K model card's §Implementation Notes ("Custom
+ * cache") keeps for hcl between calls; the turboquant-evo2-int4 model card,
+ * §"Important: a correctness fix comes with this" and §"Chunk size", requires
+ * every chunk of a prefill to continue from the previous chunk's state, and a
+ * new sequence starts from the empty one.  N >= 1 counts the state's floats
+ * per channel (pass 2N for N complex modes).  Asynchronous on `stream`.
  */
 hyena_status_t hyena_modal_state_init(float *state, int B, int D, int N, void *stream);
 

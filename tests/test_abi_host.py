@@ -81,7 +81,7 @@ def fir(lib, **kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(B=0), INVALID), (dict(L=-1), INVALID), (dict(D=0), INVALID),
     (dict(x1=None), INVALID), (dict(y=None), INVALID), (dict(lp=None), INVALID),
-    (dict(res=None), INVALID), (dict(N=0), INVALID), (dict(N=17), UNSUP),
+    (dict(res=None), INVALID), (dict(N=0), INVALID), (dict(N=65), UNSUP),
     (dict(ld_x=32), INVALID), (dict(ld_y=60), INVALID), (dict(D=60, ld_x=64, ld_y=64), ALIGN),
     (dict(ld_x=68), ALIGN), (dict(x2=A + 2), ALIGN), (dict(y=A + 8), ALIGN),
     (dict(s_in=A + 4), ALIGN), (dict(ds=A + 4), ALIGN),
@@ -110,7 +110,7 @@ def fdec(lib, x1=A, x2=A, x3=A, ld_x=64, taps=A, Ds=None, y=A, ld_y=64, hist=A, 
 
 @pytest.mark.parametrize("kw,code", [
     (dict(B=0), INVALID), (dict(state=None), INVALID), (dict(a=None), INVALID), (dict(R=None), INVALID),
-    (dict(y=None), INVALID), (dict(N=0), INVALID), (dict(N=17), UNSUP), (dict(ld_x=32), INVALID),
+    (dict(y=None), INVALID), (dict(N=0), INVALID), (dict(N=65), UNSUP), (dict(ld_x=32), INVALID),
     (dict(state=A + 4), ALIGN), (dict(x2=A + 2), ALIGN), (dict(Ds=A + 8), ALIGN), (dict(D=12, ld_x=16, ld_y=16), ALIGN),
 ])
 def test_modal_decode_rejects_bad_arguments(kw, code):
@@ -158,7 +158,7 @@ def test_packed_entry_points_check_their_own_arguments():
     same way as the plain entry point."""
     lib = hy.lib()
     assert lib.hyena_modal_long_conv_packed(A, 192, 1, A, A, None, A + 65536, 64, None, None,
-                                            1, 16, 64, 17, None, 0, None) == UNSUP
+                                            1, 16, 64, hy.MAX_MODES + 1, None, 0, None) == UNSUP
     assert lib.hyena_modal_long_conv_packed(A, 192, 64, A, A, None, A + 65536, 64, None, None,
                                             1, 16, 64, 8, None, 0, None) == WORKSPACE
     assert lib.hyena_short_conv_packed(A, 192, 8, A, None, A + 65536, 64, None, None, 1, 16, 64, 129, None) == UNSUP
@@ -190,7 +190,7 @@ def test_complex_entry_points_reject_bad_arguments():
     assert conv() == WORKSPACE
     assert conv(ws=A, ws_bytes=lib.hyena_modal_long_conv_workspace_size(1, 64, 4)) == WORKSPACE  # needs 2N slots
     assert dec(N=0) == INVALID
-    assert dec(N=9) == UNSUP
+    assert dec(N=hy.MAX_COMPLEX_MODES + 1) == UNSUP
     assert dec(s=None) == INVALID
     assert dec(s=A + 8) == ALIGN
     assert dec(ld_x=32) == INVALID

@@ -22,7 +22,7 @@ TIMEOUT = 5  # HYENA_ERR_TIMEOUT
 def test_lookback_wait_runs_out_and_is_reported():
     import torch
     import hyena_long_convolution_b200 as hy
-    B, L, D, N = 1, 4096, 64, 8  # one chain of 32 units: 16 two-unit groups
+    B, L, D, N = 1, 4096, 64, 8  # one chain of 32 units: 8 four-unit groups
     inp = make_modal_inputs(B, L, D, N, seed=77)
     x = [to_dev_bf16(inp[k]) for k in ("x1", "x2", "x3")]
     a, R, Ds = to_dev_f32(inp["log_poles"]), to_dev_f32(inp["residues"]), to_dev_f32(inp["Dskip"])

@@ -22,6 +22,8 @@ def dev(inp):
 @pytest.mark.parametrize("B,L,D,N", [
     (1, 1, 64, 8), (1, 700, 64, 8), (2, 300, 136, 3), (1, 1000, 128, 1), (3, 129, 72, 5),
     (2, 257, 24, 2), (1, 4100, 520, 8), (1, 20000, 64, 4),
+    # more than 8 complex modes (16 slots): lanes share a channel pair
+    (1, 1000, 64, 9), (2, 300, 48, 16), (1, 2100, 40, 32),
 ])
 def test_shapes_with_state(B, L, D, N):
     import torch
@@ -92,7 +94,7 @@ def test_whole_unit_chunks_are_bit_exact_and_ragged_chunks_close():
     assert rel <= STATE_TOL, rel
 
 
-@pytest.mark.parametrize("B,D,N", [(1, 64, 1), (2, 136, 5), (3, 4096, 8)])
+@pytest.mark.parametrize("B,D,N", [(1, 64, 1), (2, 136, 5), (3, 4096, 8), (1, 64, 9), (2, 96, 32)])
 def test_decode_step_matches_oracle_and_prefill(B, D, N):
     import torch
     import hyena_long_convolution_b200 as hy

@@ -15,7 +15,8 @@ from .helpers import assert_close, bits_of, from_dev_bf16, metrics, to_dev_bf16,
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("B,D,N", [(1, 64, 1), (2, 136, 5), (3, 200, 8), (1, 4096, 16)])
+@pytest.mark.parametrize("B,D,N", [(1, 64, 1), (2, 136, 5), (3, 200, 8), (1, 4096, 16), (1, 64, 17),
+                                   (2, 136, 32), (1, 200, 50), (2, 4096, 64)])
 def test_modal_decode_step_matches_oracle_and_prefill(B, D, N):
     import torch
     import hyena_long_convolution_b200 as hy

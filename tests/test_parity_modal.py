@@ -79,6 +79,9 @@ def test_modal_1k_with_state_and_direct_form():
 @pytest.mark.parametrize("B,L,D,N", [
     (1, 1, 64, 16), (1, 2, 8, 1), (2, 127, 72, 3), (1, 128, 64, 8), (2, 129, 136, 16),
     (3, 1000, 200, 5), (1, 2048, 64, 16), (2, 4100, 520, 12), (1, 40000, 64, 4), (2, 300, 24, 4),
+    # more than 16 modes: two or four lanes share a channel pair, narrower chains
+    (1, 1, 32, 17), (2, 1000, 72, 20), (1, 4100, 96, 32), (1, 129, 16, 33), (2, 700, 40, 48),
+    (1, 3000, 64, 64), (1, 64, 8, 64),
 ])
 def test_shapes_ragged(B, L, D, N):
     inp = make_modal_inputs(B, L, D, N, seed=B * 1000 + L + D + N)
@@ -146,3 +149,21 @@ def test_special_values_propagate():
     assert np.array_equal(b0[:, :300], b1[:, :300])
     assert np.array_equal(b0[:, :, :5], b1[:, :, :5]) and np.array_equal(b0[:, :, 6:], b1[:, :, 6:])
     assert not np.all(np.isfinite(from_dev_bf16(y1)[0, 300:, 5]))
+
+
+@pytest.mark.parametrize("N", [32, 64])
+def test_many_modes_8k_by_1024_channels(N):
+    # 1 <= N <= 64 real modes at a longer size: every element against the oracle
+    inp = make_modal_inputs(1, 8192, 1024, N, seed=N)
+    S = np.random.default_rng(N).standard_normal((1, 1024, N))
+    check(inp, S)
+
+
+@pytest.mark.parametrize("N", [20, 64])
+def test_many_modes_whole_unit_chunks_are_bit_exact(N):
+    inp = make_modal_inputs(1, 1024, 64, N, seed=7 + N)
+    S0 = np.random.default_rng(9).standard_normal((1, 64, N))
+    y1, s1 = check(inp, S0)
+    yc, sc = check(inp, S0, chunks=[256, 128, 640])
+    assert np.array_equal(bits_of(yc), bits_of(y1))
+    assert np.array_equal(sc.cpu().numpy(), s1.cpu().numpy())

@@ -127,6 +127,8 @@ def measured_peaks():
 
 KERNEL_SOURCES = {
     "modal": ("hyena_long_convolution_b200/csrc/modal_scan.cu",
+              "hyena_long_convolution_b200/csrc/modal_scan_wide.cu",
+              "hyena_long_convolution_b200/csrc/modal_synth.cu",
               "hyena_long_convolution_b200/csrc/hyena_device.cuh",
               "hyena_long_convolution_b200/csrc/hyena_internal.h"),
     "fir": ("hyena_long_convolution_b200/csrc/short_conv.cu",

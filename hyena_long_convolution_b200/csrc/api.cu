@@ -94,6 +94,22 @@ bool encode_x_map(CUtensorMap *m, const XSource &xs, int k, int B, int L, int D,
     return r == CUDA_SUCCESS;
 }
 
+// 2-D fp32 tensor map over the modal coefficient table [4 NPT + 1][Dp]: box
+// of `width` columns (one chain) x rows [0, 2 NPT + 1) (p, residues, Dskip).
+bool encode_coef_map(CUtensorMap *m, void *table, int Dp, int NPT, int width)
+{
+    std::call_once(g_encode_once, resolve_encode);
+    if (g_encode == nullptr) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(Dp), static_cast<cuuint64_t>(modal_coef_rows(NPT))};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(Dp) * 4};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(width), static_cast<cuuint32_t>(2 * NPT + 1)};
+    cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, table, dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 hyena_status_t check_x(const void *x1, const void *x2, const void *x3, long long ld_x, const void *y,
@@ -302,20 +318,35 @@ hyena_status_t modal_long_conv_impl(const XSource &xs, const float *log_poles, c
     sy.Dp = lay.Dp;
     sy.coef = reinterpret_cast<float *>(ws + lay.off_coef);
 
-    ModalMaps maps;
-    const int width = MCH / lay.LPC;  // channels per chain
-    if (!encode_x_map(&maps.a1, xs, 0, B, L, D, MA_ROWS, width) ||
-        !encode_x_map(&maps.c1, xs, 0, B, L, D, MC_ROWS, width))
-        return HYENA_ERR_CUDA;
-    if (xs.triples) {
-        maps.a2 = maps.a1;
-        maps.c2 = maps.c3 = maps.c1;
-    } else if (!encode_x_map(&maps.a2, xs, 1, B, L, D, MA_ROWS, width) ||
-               !encode_x_map(&maps.c2, xs, 1, B, L, D, MC_ROWS, width) ||
-               !encode_x_map(&maps.c3, xs, 2, B, L, D, MC_ROWS, width)) {
-        return HYENA_ERR_CUDA;
+    const int ns = launch_modal_synth(sy, lay.NP, cx, s);
+    if (ns < 0) return HYENA_ERR_CUDA;
+    int n = -1;
+    if (lay.LPC == 1) {
+        CUtensorMap m1, m2, m3;
+        if (!encode_x_map(&m1, xs, 0, B, L, D, MCK)) return HYENA_ERR_CUDA;
+        if (xs.triples)
+            m2 = m3 = m1;
+        else if (!encode_x_map(&m2, xs, 1, B, L, D, MCK) || !encode_x_map(&m3, xs, 2, B, L, D, MCK))
+            return HYENA_ERR_CUDA;
+        n = launch_modal_narrow(m1, m2, m3, a, lay.NP, xs.triples, cx, s);
+    } else {
+        ModalMaps maps;
+        const int width = MCH / lay.LPC;  // channels per chain
+        if (!encode_x_map(&maps.a1, xs, 0, B, L, D, MA_ROWS, width) ||
+            !encode_x_map(&maps.c1, xs, 0, B, L, D, MC_ROWS, width))
+            return HYENA_ERR_CUDA;
+        if (xs.triples) {
+            maps.a2 = maps.a1;
+            maps.c2 = maps.c3 = maps.c1;
+        } else if (!encode_x_map(&maps.a2, xs, 1, B, L, D, MA_ROWS, width) ||
+                   !encode_x_map(&maps.c2, xs, 1, B, L, D, MC_ROWS, width) ||
+                   !encode_x_map(&maps.c3, xs, 2, B, L, D, MC_ROWS, width)) {
+            return HYENA_ERR_CUDA;
+        }
+        if (!encode_coef_map(&maps.coef, ws + lay.off_coef, lay.Dp, lay.NP, width)) return HYENA_ERR_CUDA;
+        n = launch_modal_wide(maps, a, lay.NP, xs.triples, cx, s);
     }
-    const int n = launch_modal(maps, a, sy, lay.NP, xs.triples, cx, s);
+    if (n >= 0) n += ns;
     if (n < 0) return HYENA_ERR_CUDA;
     g_last_launches = n;
     return HYENA_OK;
@@ -558,10 +589,18 @@ hyena_status_t hyena_workspace_check(void *workspace, void *stream)
 {
     if (workspace == nullptr) return HYENA_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (cudaStreamSynchronize(s) != cudaSuccess) return HYENA_ERR_CUDA;
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "workspace check: stream synchronize");
+        return HYENA_ERR_CUDA;
+    }
     unsigned int err = 0;
     unsigned int *hdr = static_cast<unsigned int *>(workspace);
-    if (cudaMemcpy(&err, hdr + 2, sizeof err, cudaMemcpyDeviceToHost) != cudaSuccess) return HYENA_ERR_CUDA;
+    e = cudaMemcpy(&err, hdr + 2, sizeof err, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) {
+        record_cuda_error(e, "workspace check: read error word");
+        return HYENA_ERR_CUDA;
+    }
     if (err != 0u) {
         if (cudaMemset(hdr + 2, 0, sizeof err) != cudaSuccess) return HYENA_ERR_CUDA;
         return HYENA_ERR_TIMEOUT;

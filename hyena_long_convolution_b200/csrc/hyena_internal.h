@@ -46,9 +46,8 @@ __host__ __device__ __forceinline__ long long x_col(int c, int group)
 // A chain is the sequence of MCH channels of one batch row over time.  A unit
 // is MT consecutive tokens of a chain: the carry from one unit to the next
 // follows one canonical fp32 recurrence, so feeding a sequence in chunks of
-// whole units reproduces the single pass bit for bit.  A group is MGMAX
-// consecutive units of a chain, the work item one CTA takes at a time: one
-// aggregate warp per unit and one output warp per half unit (MH tokens).
+// whole units reproduces the single pass bit for bit.  A group is up to MGMAX
+// consecutive units of a chain, the work item one CTA takes at a time.
 // Up to 16 mode slots per lane: lane l of a warp owns the channel pair 2l,
 // 2l+1 of a 64-channel chain and all its (padded) mode slots.  With 32 or 64
 // slots, LPC = 2 or 4 lanes share a channel pair, each owning 16 consecutive
@@ -110,24 +109,39 @@ struct ModalSynthArgs {
     float *coef;
 };
 
-// Rows of the tensor-map boxes the scan kernel reads: aggregate warps take
-// MA_ROWS tokens per chunk (x1, x2), output warps MC_ROWS (x1, x2, x3).
+// Up to 16 mode slots (the common case) the scan runs as the two-CTAs-per-SM
+// kernel of modal_scan.cu: each compute warp sweeps its unit's aggregate and
+// then its outputs, streaming chunks of MCK rows x MCH channels of x1/x2 (and
+// x3).  With 32 or 64 slots it runs as the warp-specialised kernel of
+// modal_scan_wide.cu (chains of MCH / LPC channels; aggregate warps read
+// chunks of MA_ROWS rows, output warps chunks of MC_ROWS rows).
+constexpr int MCK = 16;
 constexpr int MA_ROWS = 16;
-constexpr int MC_ROWS = 8;
+constexpr int MC_ROWS = 16;
 
-// Launches the coefficient-synthesis kernel and the scan kernel; returns the
-// number of launches enqueued or a negative value on a CUDA error.  The 4-D
-// tensor maps [B][L][groups][group] cover x1, x2 (a1, a2: boxes of MA_ROWS
-// rows x MCH channels) and x1, x2, x3 (c1..c3: boxes of MC_ROWS rows); with
-// `triples` a1 and c1 alone cover the interleaved rows (boxes of 3 MCH
-// elements per row) and the others are unused.  With `cx` the N of the
-// arguments counts mode slots, two per complex mode (state [B][D][N/2][2] =
-// [B][D][N]).
+// Launches the coefficient-synthesis kernel for NPT padded slots; returns the
+// number of launches enqueued or a negative value on a CUDA error.  With `cx`
+// the N of the arguments counts mode slots, two per complex mode.
+int launch_modal_synth(const ModalSynthArgs &s, int NPT, bool cx, cudaStream_t st);
+
+// The scan for NP <= 16 padded slots: three 4-D tensor maps [B][L][groups][group]
+// over x1, x2, x3 with boxes of MCK rows x MCH channels; with `triples` the
+// first map alone covers the interleaved rows (boxes of MCK rows x 3 MCH
+// elements) and the other two are unused.  With `cx` the N of the arguments
+// counts mode slots, two per complex mode (state [B][D][N/2][2] = [B][D][N]).
+// Returns the number of launches or a negative value on a CUDA error.
+int launch_modal_narrow(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3, ModalArgs a, int NP,
+                        bool triples, bool cx, cudaStream_t st);
+
+// The scan for NPT = 32 or 64 padded slots.  Maps over x1, x2 (a1, a2: boxes
+// of MA_ROWS rows x chain width) and x1, x2, x3 (c1..c3: boxes of MC_ROWS
+// rows); with `triples` a1 and c1 alone cover the interleaved rows.  coef: a
+// 2-D map over the coefficient table [4NPT+1][Dp] fp32, box of one chain's
+// columns x rows [0, 2NPT+1) (p, residues, Dskip).
 struct ModalMaps {
-    CUtensorMap a1, a2, c1, c2, c3;
+    CUtensorMap a1, a2, c1, c2, c3, coef;
 };
-int launch_modal(const ModalMaps &maps, ModalArgs a, const ModalSynthArgs &s, int NPT, bool triples, bool cx,
-                 cudaStream_t st);
+int launch_modal_wide(const ModalMaps &maps, ModalArgs a, int NPT, bool triples, bool cx, cudaStream_t st);
 
 // ---------------------------------------------------------------- short FIR
 constexpr int FCH = 64;   // channels per CTA

@@ -290,6 +290,8 @@ hyena_status_t modal_long_conv_impl(const XSource &xs, const float *log_poles, c
 
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     ModalArgs a{};
+    a.x1 = xs.x[0];
+    a.x2 = xs.x[1];
     a.x3 = xs.x[2];
     a.ld_x = xs.ld;
     a.group = xs.group;
@@ -328,7 +330,9 @@ hyena_status_t modal_long_conv_impl(const XSource &xs, const float *log_poles, c
             m2 = m3 = m1;
         else if (!encode_x_map(&m2, xs, 1, B, L, D, MCK) || !encode_x_map(&m3, xs, 2, B, L, D, MCK))
             return HYENA_ERR_CUDA;
-        n = launch_modal_narrow(m1, m2, m3, a, lay.NP, xs.triples, cx, s);
+        n = modal_short_path(B, L, D, lay.NP, xs.triples)
+                ? launch_modal_short(m1, m2, m3, a, lay.NP, xs.triples, cx, s)
+                : launch_modal_narrow(m1, m2, m3, a, lay.NP, xs.triples, cx, s);
     } else {
         ModalMaps maps;
         const int width = MCH / lay.LPC;  // channels per chain

@@ -83,7 +83,7 @@ struct ModalLayout {
 ModalLayout modal_layout(int B, int D, int N);
 
 struct ModalArgs {
-    const uint16_t *x3;
+    const uint16_t *x1, *x2, *x3;  // x[0..2] of the input source (see x_col)
     long long ld_x;
     int group;                  // channel group of the inputs (see x_col)
     uint16_t *y;
@@ -141,6 +141,16 @@ int launch_modal_narrow(const CUtensorMap &m1, const CUtensorMap &m2, const CUte
 struct ModalMaps {
     CUtensorMap a1, a2, c1, c2, c3, coef;
 };
+// Short sequences: up to 16 slots, at most MSHORT_UNITS units per chain whose
+// x1/x2 rows (B L D 4 bytes, 6 for triples) fit in MSHORT_L2_BYTES of L2.
+// There the scan runs as two plain passes over all units at once (aggregates,
+// then carries and outputs) with the look-back kernel's arithmetic.
+constexpr int MSHORT_UNITS = 24;
+constexpr long long MSHORT_L2_BYTES = 48ll << 20;
+bool modal_short_path(int B, int L, int D, int NP, bool triples);
+int launch_modal_short(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3, const ModalArgs &a,
+                       int NP, bool triples, bool cx, cudaStream_t st);
+
 int launch_modal_wide(const ModalMaps &maps, ModalArgs a, int NPT, bool triples, bool cx, cudaStream_t st);
 
 // ---------------------------------------------------------------- short FIR

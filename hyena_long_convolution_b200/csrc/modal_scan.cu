@@ -685,6 +685,313 @@ int launch_narrow_layout(const CUtensorMap &m1, const CUtensorMap &m2, const CUt
     }
 }
 
+// ------------------------------------------------------------------ short sequences
+// With few units per chain the look-back kernel leaves most sub-partitions
+// idle and its chain of look-backs is most of the launch.  There two plain
+// passes over all units at once do better:
+//   pass 1  one warp per unit sweeps the unit's aggregate A_j from a zero
+//           start into the chain's slot area (the warp of unit 0 also copies
+//           state_in there as C_0, so that pass 2 never reads a state_in
+//           that aliases state_out);
+//   pass 2  one warp per unit forms its carry C_j by folding C_0 and
+//           A_0 .. A_{j-1} forward in order and sweeps the unit's outputs;
+//           x1/x2 come back from L2.
+// Every value is formed by the look-back kernel's operations in the same
+// order (aggregate sweep, canonical carry chain, output sweep), so the two
+// paths give the same bits and a chunked sequence may mix them.
+//
+// Each warp requests all of its unit's rows with TMA at once (one barrier per
+// chunk of MCK rows), so a launch keeps every unit's bytes in flight.  The
+// coefficient kernel and the two passes are chained by programmatic dependent
+// launch: a pass issues its row loads (inputs no kernel of the call writes)
+// before it waits for the previous kernel's results.
+constexpr int kShortWarps = 2;          // units per CTA
+constexpr int kShortChunks = MT / MCK;  // chunks of MCK rows per unit
+static_assert(MSHORT_UNITS + 1 <= MRING * (MGMAX + 1), "a chain's slot area holds C_0 and every unit's aggregate");
+
+template <int kTensors>
+struct ShortSmem {
+    uint32_t chunk[kShortWarps][kShortChunks][kTensors][kChunkWords];
+    uint64_t full[kShortWarps][kShortChunks];
+};
+static_assert(sizeof(uint32_t) * 2 * kChunkWords % 128 == 0, "TMA destinations stay 128-byte aligned");
+
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+struct ShortPos {
+    int chain, b, cb, j, c0, t0, nvalid;
+    bool ch_ok;
+};
+
+// Position of this warp's unit; false past the last unit.
+__device__ __forceinline__ bool short_pos(const ModalArgs &A, ShortPos &q)
+{
+    const long long u = static_cast<long long>(blockIdx.x) * kShortWarps + (threadIdx.x >> 5);
+    const long long chains = static_cast<long long>(A.B) * A.nCB;
+    if (u >= chains * A.units) return false;
+    q.chain = static_cast<int>(u / A.units);
+    q.j = static_cast<int>(u - static_cast<long long>(q.chain) * A.units);
+    q.b = q.chain / A.nCB;
+    q.cb = q.chain % A.nCB;
+    q.c0 = q.cb * MCH + 2 * (threadIdx.x & 31);
+    q.ch_ok = q.c0 < A.D;
+    q.t0 = q.j * MT;
+    q.nvalid = min(MT, A.L - q.t0);
+    return true;
+}
+
+// Lane 0 requests chunks 0 .. nchunks-1 of the warp's unit: x1/x2 (and x3
+// with kX3), or the triples box, one barrier per chunk.  Rows past L and
+// channels past D land as zeros, as in the look-back kernel.  The warp waits
+// for every chunk it requested before it leaves.
+template <int kTensors, bool kTri, bool kX3>
+__device__ __forceinline__ void short_issue(ShortSmem<kTensors> &sm, int w, int nchunks, const ShortPos &q,
+                                            const ModalArgs &A, const CUtensorMap *tm1, const CUtensorMap *tm2,
+                                            const CUtensorMap *tm3)
+{
+    if ((threadIdx.x & 31) == 0) {
+#pragma unroll
+        for (int i = 0; i < kShortChunks; ++i) mbar_init(&sm.full[w][i], 1);
+        fence_mbar_init();
+        const int ch = q.cb * MCH;
+        const int cx = kTri ? 3 * ch : ch % A.group;
+        const int cg = kTri ? 0 : ch / A.group;
+#pragma unroll 1
+        for (int i = 0; i < nchunks; ++i) {
+            uint64_t *bar = &sm.full[w][i];
+            const int row = q.t0 + i * MCK;
+            if constexpr (kTri) {
+                mbar_arrive_expect_tx(bar, 3 * kChunkBytes);
+                tma_load_4d(sm.chunk[w][i][0], tm1, bar, cx, 0, row, q.b);
+            } else {
+                mbar_arrive_expect_tx(bar, (kX3 ? 3 : 2) * kChunkBytes);
+                tma_load_4d(sm.chunk[w][i][0], tm1, bar, cx, cg, row, q.b);
+                tma_load_4d(sm.chunk[w][i][1], tm2, bar, cx, cg, row, q.b);
+                if constexpr (kX3) tma_load_4d(sm.chunk[w][i][2], tm3, bar, cx, cg, row, q.b);
+            }
+        }
+    }
+    __syncwarp();
+}
+
+// Slot of unit j's aggregate (j == units: C_0), this lane's channel pair.
+template <int NP>
+__device__ __forceinline__ float *short_unit_slot(const ModalArgs &A, int chain, int j)
+{
+    const size_t slot_floats = static_cast<size_t>(MGMAX + 1) * NP * MCH;
+    return A.slots + static_cast<size_t>(chain) * MRING * slot_floats + static_cast<size_t>(j) * NP * MCH +
+           2 * (threadIdx.x & 31);
+}
+
+template <int NP, bool kTri, bool kCx>
+__global__ void __launch_bounds__(32 * kShortWarps) modal_short_agg_kernel(const __grid_constant__ CUtensorMap tm1,
+                                                                          const __grid_constant__ CUtensorMap tm2,
+                                                                          const ModalArgs A)
+{
+    constexpr int kT = kTri ? 3 : 2;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    ShortSmem<kT> &sm = *reinterpret_cast<ShortSmem<kT> *>(smem_raw);
+    pdl_launch_dependents();
+    ShortPos q;
+    if (!short_pos(A, q)) return;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // all chunks: the aggregate runs over the zero rows past L as well
+    short_issue<kT, kTri, false>(sm, w, kShortChunks, q, A, &tm1, &tm2, nullptr);
+    pdl_wait();  // the coefficient table, and the slot area a previous call read
+    if (q.j == 0) {
+        float *c0slot = short_unit_slot<NP>(A, q.chain, A.units);
+#pragma unroll
+        for (int n = 0; n < NP; ++n) {
+            float2 v = make_float2(0.f, 0.f);
+            if (A.state_in != nullptr && n < A.N && q.ch_ok) {
+                v.x = A.state_in[(static_cast<size_t>(q.b) * A.D + q.c0) * A.N + n];
+                v.y = A.state_in[(static_cast<size_t>(q.b) * A.D + q.c0 + 1) * A.N + n];
+            }
+            *reinterpret_cast<float2 *>(c0slot + n * MCH) = v;
+        }
+    }
+    float2 p[NP], s[NP];
+    load_rows<NP>(p, A.coef, 0, A.Dp, q.c0);
+#pragma unroll
+    for (int n = 0; n < NP; ++n) s[n] = make_float2(0.f, 0.f);
+    for (int i = 0; i < kShortChunks; ++i) {
+        (void)mbar_wait_tiles(&sm.full[w][i], 0, A.hdr);
+        if constexpr (kTri)
+            sweep_a_chunk_tri<NP, kCx>(s, p, &sm.chunk[w][i][0][0] + 3 * lane);
+        else
+            sweep_a_chunk<NP, kCx>(s, p, sm.chunk[w][i][0] + lane, sm.chunk[w][i][1] + lane);
+    }
+    float *slot = short_unit_slot<NP>(A, q.chain, q.j);
+#pragma unroll
+    for (int n = 0; n < NP; ++n) *reinterpret_cast<float2 *>(slot + n * MCH) = s[n];
+}
+
+template <int NP, bool kTri, bool kCx>
+__global__ void __launch_bounds__(32 * kShortWarps) modal_short_out_kernel(const __grid_constant__ CUtensorMap tm1,
+                                                                          const __grid_constant__ CUtensorMap tm2,
+                                                                          const __grid_constant__ CUtensorMap tm3,
+                                                                          const ModalArgs A)
+{
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    ShortSmem<3> &sm = *reinterpret_cast<ShortSmem<3> *>(smem_raw);
+    ShortPos q;
+    if (!short_pos(A, q)) return;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nchunks = (q.nvalid + MCK - 1) / MCK;  // the chunks holding rows inside L
+    short_issue<3, kTri, true>(sm, w, nchunks, q, A, &tm1, &tm2, &tm3);
+    pdl_wait();  // the aggregates and C_0 of pass 1
+    pdl_launch_dependents();
+
+    // ---------------- the carry into unit j: the canonical chain
+    float2 C[NP];
+    {
+        float2 pT[NP];
+        load_rows<NP>(pT, A.coef, 2 * NP + 1, A.Dp, q.c0);
+        const float *c0slot = short_unit_slot<NP>(A, q.chain, A.units);
+#pragma unroll
+        for (int n = 0; n < NP; ++n) C[n] = __ldcg(reinterpret_cast<const float2 *>(c0slot + n * MCH));
+        const float *base = short_unit_slot<NP>(A, q.chain, 0);
+        int jj = 0;
+        for (; jj + 2 <= q.j; jj += 2) {
+            // two units' aggregates in flight at once
+            float2 a[NP], b2[NP];
+#pragma unroll
+            for (int n = 0; n < NP; ++n) {
+                a[n] = __ldcg(reinterpret_cast<const float2 *>(base + (static_cast<size_t>(jj) * NP + n) * MCH));
+                b2[n] = __ldcg(reinterpret_cast<const float2 *>(base + (static_cast<size_t>(jj + 1) * NP + n) * MCH));
+            }
+            modes_carry<NP, kCx>(C, pT, a);
+            modes_carry<NP, kCx>(C, pT, b2);
+        }
+        if (jj < q.j) {
+            float2 a[NP];
+#pragma unroll
+            for (int n = 0; n < NP; ++n)
+                a[n] = __ldcg(reinterpret_cast<const float2 *>(base + (static_cast<size_t>(jj) * NP + n) * MCH));
+            modes_carry<NP, kCx>(C, pT, a);
+        }
+        // A sequence ending on a unit boundary takes its final state from the
+        // canonical chain, C_units.
+        if ((A.L % MT) == 0 && q.j == A.units - 1 && A.state_out != nullptr && q.ch_ok) {
+            float2 a[NP], Cn[NP];
+#pragma unroll
+            for (int n = 0; n < NP; ++n) {
+                a[n] = __ldcg(reinterpret_cast<const float2 *>(base + (static_cast<size_t>(q.j) * NP + n) * MCH));
+                Cn[n] = C[n];
+            }
+            modes_carry<NP, kCx>(Cn, pT, a);
+#pragma unroll
+            for (int n = 0; n < NP; ++n) {
+                if (n < A.N) {
+                    A.state_out[(static_cast<size_t>(q.b) * A.D + q.c0) * A.N + n] = Cn[n].x;
+                    A.state_out[(static_cast<size_t>(q.b) * A.D + q.c0 + 1) * A.N + n] = Cn[n].y;
+                }
+            }
+        }
+    }
+
+    // ---------------- outputs of the unit from its carry
+    float2 p[NP], R[NP];
+    load_rows<NP>(p, A.coef, 0, A.Dp, q.c0);
+    load_rows<NP>(R, A.coef, NP, A.Dp, q.c0);
+    const float2 dsk = ldg_f2(A.coef + static_cast<size_t>(2 * NP) * A.Dp + q.c0);
+    uint32_t *yrow = reinterpret_cast<uint32_t *>(A.y + (static_cast<size_t>(q.b) * A.L + q.t0) * A.ld_y + q.c0);
+    const size_t ystride = static_cast<size_t>(A.ld_y) / 2;  // in 32-bit words
+    for (int i = 0; i < nchunks; ++i) {
+        (void)mbar_wait_tiles(&sm.full[w][i], 0, A.hdr);
+        const int base = i * MCK;
+        uint32_t *yc = yrow + static_cast<size_t>(base) * ystride;
+        if (base + MCK <= q.nvalid) {
+#pragma unroll
+            for (int r = 0; r < MCK; ++r) {
+                float2 v, x3;
+                chunk_row<kTri>(sm.chunk[w][i], lane, r, v, x3);
+                sweep_c_token<NP, kCx>(C, p, R, dsk, v, x3, yc + r * ystride, q.ch_ok);
+            }
+        } else {
+            for (int r = 0; r < MCK && base + r < q.nvalid; ++r) {
+                float2 v, x3;
+                chunk_row<kTri>(sm.chunk[w][i], lane, r, v, x3);
+                sweep_c_token<NP, kCx>(C, p, R, dsk, v, x3, yc + r * ystride, q.ch_ok);
+            }
+        }
+    }
+    // A ragged last unit: the final state is the recurrence state after token L-1.
+    if (A.state_out != nullptr && q.ch_ok && (A.L % MT) != 0 && q.j == A.units - 1) {
+#pragma unroll
+        for (int n = 0; n < NP; ++n) {
+            if (n < A.N) {
+                A.state_out[(static_cast<size_t>(q.b) * A.D + q.c0) * A.N + n] = C[n].x;
+                A.state_out[(static_cast<size_t>(q.b) * A.D + q.c0 + 1) * A.N + n] = C[n].y;
+            }
+        }
+    }
+}
+
+template <class Kernel, class... Args>
+cudaError_t launch_dependent(Kernel kernel, unsigned int grid, int threads, size_t smem, cudaStream_t st,
+                             Args... args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+template <int NP, bool kTri, bool kCx>
+int launch_short_np(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3, const ModalArgs &a,
+                    cudaStream_t st)
+{
+    static int configured_device = -1;
+    int dev = 0;
+    HYENA_TRY(cudaGetDevice(&dev), "cudaGetDevice");
+    constexpr size_t smem_agg = sizeof(ShortSmem<kTri ? 3 : 2>);
+    constexpr size_t smem_out = sizeof(ShortSmem<3>);
+    auto agg = modal_short_agg_kernel<NP, kTri, kCx>;
+    auto out = modal_short_out_kernel<NP, kTri, kCx>;
+    if (configured_device != dev) {
+        HYENA_TRY(cudaFuncSetAttribute(agg, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_agg)),
+                  "modal scan (short): set max dynamic shared memory");
+        HYENA_TRY(cudaFuncSetAttribute(out, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_out)),
+                  "modal scan (short): set max dynamic shared memory");
+        configured_device = dev;
+    }
+    const long long units = static_cast<long long>(a.B) * a.nCB * a.units;
+    const unsigned int grid = static_cast<unsigned int>((units + kShortWarps - 1) / kShortWarps);
+    HYENA_TRY(launch_dependent(agg, grid, 32 * kShortWarps, smem_agg, st, m1, m2, a),
+              "modal scan (short): aggregate pass launch");
+    HYENA_TRY(launch_dependent(out, grid, 32 * kShortWarps, smem_out, st, m1, m2, m3, a),
+              "modal scan (short): output pass launch");
+    return 2;
+}
+
+template <bool kTri, bool kCx>
+int launch_short_layout(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3, const ModalArgs &a,
+                        int NP, cudaStream_t st)
+{
+    switch (NP) {
+        case 4: return launch_short_np<4, kTri, kCx>(m1, m2, m3, a, st);
+        case 8: return launch_short_np<8, kTri, kCx>(m1, m2, m3, a, st);
+        case 16: return launch_short_np<16, kTri, kCx>(m1, m2, m3, a, st);
+        default: return -1;
+    }
+}
+
 }  // namespace
 
 int launch_modal_narrow(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3, ModalArgs a, int NP,
@@ -695,6 +1002,24 @@ int launch_modal_narrow(const CUtensorMap &m1, const CUtensorMap &m2, const CUte
                   : launch_narrow_layout<true, false>(m1, m2, m3, a, NP, st);
     return cx ? launch_narrow_layout<false, true>(m1, m2, m3, a, NP, st)
               : launch_narrow_layout<false, false>(m1, m2, m3, a, NP, st);
+}
+
+bool modal_short_path(int B, int L, int D, int NP, bool triples)
+{
+    if (NP > 16 || L < 1) return false;
+    const long long units = (static_cast<long long>(L) + MT - 1) / MT;
+    const long long bytes = static_cast<long long>(B) * L * D * (triples ? 6 : 4);
+    return units <= MSHORT_UNITS && bytes <= MSHORT_L2_BYTES;
+}
+
+int launch_modal_short(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3, const ModalArgs &a,
+                       int NP, bool triples, bool cx, cudaStream_t st)
+{
+    if (triples)
+        return cx ? launch_short_layout<true, true>(m1, m2, m3, a, NP, st)
+                  : launch_short_layout<true, false>(m1, m2, m3, a, NP, st);
+    return cx ? launch_short_layout<false, true>(m1, m2, m3, a, NP, st)
+              : launch_short_layout<false, false>(m1, m2, m3, a, NP, st);
 }
 
 }  // namespace hyena

@@ -15,6 +15,9 @@ namespace {
 template <int NPT>
 __global__ void modal_synth_kernel(const ModalSynthArgs S)
 {
+    // a pass launched as this kernel's dependent may start its input loads
+    // now; it waits for this grid before it reads the table
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int idx = blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= NPT * S.Dp) return;
     const int n = idx / S.Dp;
@@ -38,6 +41,7 @@ template <int NPT>
 __global__ void modal_csynth_kernel(const ModalSynthArgs S)
 {
     static_assert(MT == 128 && MH == 64, "p^MH and p^MT by squarings");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int idx = blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= NPT * S.Dp) return;
     const int n = idx / S.Dp;

@@ -115,6 +115,18 @@ def flops_per_chtok(wl):
     return 2 * wl["K"] + 4
 
 
+def kernel_fma_per_chtok(wl):
+    """FP32 FMA-pipe operations per channel-token that the kernels issue at
+    the least: the modal scan sweeps every unit twice (the aggregate, N FMAs
+    per real mode slot, then the outputs, 2N), forms v = x1 x2 in both sweeps
+    and applies the gate and the skip (3N + 4; complex modes: 4 per mode in
+    the aggregate, 6 in the output sweep); the FIR kernels K FMAs plus v, the
+    gate and the skip."""
+    if wl["kind"] == "modal":
+        return (10 * wl["N"] if wl.get("cx") else 3 * wl["N"]) + 4
+    return wl["K"] + 3
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -633,8 +645,13 @@ def run_gpu(args, wl):
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "peak_source": f"{peak_kind} hbm_gbs (copy)"}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    # The kernels' own arithmetic floor: their FMA-pipe work at the SIMT peak
+    # (a step cannot beat it however well its memory traffic is hidden).
+    fma_floor_ms = kernel_fma_per_chtok(wl) * chtok / (alu_peak * 1e12 / 2) * 1e3 if not wl.get("decode") else None
     roof.update({"traffic": traffic, "algorithmic_bytes_per_step": step_bytes,
-                 "hbm_frac": achieved / peak, "kernel_ms_min": per_sorted[0], "kernel_ms_avg": avg_ms})
+                 "hbm_frac": achieved / peak, "kernel_ms_min": per_sorted[0], "kernel_ms_avg": avg_ms,
+                 "fma_floor_ms": fma_floor_ms,
+                 "fma_floor_frac": (fma_floor_ms / avg_ms) if fma_floor_ms else None})
 
     line = {
         "metric": METRIC,

@@ -73,7 +73,9 @@ def assert_close(y, ref, what="y", per_channel=False):
         rms_c = np.sqrt(np.mean(r ** 2, axis=0))
         worst = float(np.max(np.max(excess, axis=0) / np.maximum(rms_c, 1e-300)))
         assert worst <= MAX_ABS_TOL, f"{what}: per-channel max-abs {worst:.3e} > {MAX_ABS_TOL}"
+        print(f"{what}: rel-L2 {rel:.3e}, max-abs/rms {mabs:.3e}, per-channel max-abs worst {worst:.3e}")
         return rel, worst
+    print(f"{what}: rel-L2 {rel:.3e}, max-abs/rms {mabs:.3e}")
     return rel, mabs
 
 

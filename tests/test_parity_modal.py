@@ -49,11 +49,11 @@ def run_gpu(inp, state_in=None, chunks=None, ld_pad=0, alias=False):
     return y, S_out
 
 
-def check(inp, state_in=None, **kw):
+def check(inp, state_in=None, what="y", **kw):
     y, S = run_gpu(inp, state_in, **kw)
     ref_y, ref_S = oracle.modal_recurrence(inp["x1"], inp["x2"], inp["x3"], inp["log_poles"],
                                            inp["residues"], inp["Dskip"], state_in)
-    assert_close(from_dev_bf16(y), ref_y)
+    assert_close(from_dev_bf16(y), ref_y, what)
     rel, _ = metrics(S.cpu().numpy().astype(np.float64), ref_S)
     assert rel <= STATE_TOL, f"state rel-L2 {rel:.3e}"
     return y, S
@@ -62,7 +62,7 @@ def check(inp, state_in=None, **kw):
 def test_modal_1k_full():
     c = WORKLOAD_SHAPES["modal_1k"]
     inp = make_modal_inputs(c["B"], c["L"], c["D"], c["N"], c["seed"])
-    check(inp)
+    check(inp, what="modal 1K (B=1 L=1024 D=64 N=8)")
 
 
 def test_modal_1k_with_state_and_direct_form():

@@ -526,6 +526,9 @@ def time_steps(step, steps, warmup, device):
     return per
 
 
+E2E_CHUNK = 2048  # tokens per chunk of the host-buffer entry point (16 units)
+
+
 def e2e_leg(wl, host, dev, device, steps, warmup):
     """Same metric through the public binding with pinned host buffers: every
     step copies x1/x2/x3 (and the filter parameters) host->device, runs the
@@ -538,10 +541,17 @@ def e2e_leg(wl, host, dev, device, steps, warmup):
         return t.pin_memory()
 
     hx = {k: pin(v) for k, v in host.items()}
-    dx = {k: torch.empty(v.shape, dtype=v.dtype, device=device) for k, v in hx.items()}
+    # The real-mode prefill streams its host buffers through the library's
+    # host-buffer entry point (chunks of whole units, copies in both
+    # directions overlapping the scan); everything else copies them here.
+    streamed = wl["kind"] == "modal" and not (wl.get("cx") or wl.get("group") or wl.get("decode"))
+    on_host = ("x1", "x2", "x3") if streamed else ()
+    dx = {k: torch.empty(v.shape, dtype=v.dtype, device=device) for k, v in hx.items() if k not in on_host}
     y_host = torch.empty((wl["B"], wl["L"], wl["D"]), dtype=torch.int16).pin_memory()
     B, L, D = wl["B"], wl["L"], wl["D"]
     y = torch.empty((B, L, D), dtype=torch.bfloat16, device=device)
+    if streamed:
+        hws = hy.HostWorkspace(B, D, wl["N"], chunk=E2E_CHUNK, device=device)
     if wl["kind"] == "modal":
         cx = bool(wl.get("cx"))
         ws = hy.ModalWorkspace(B, D, (2 if cx else 1) * wl["N"], device=device)
@@ -550,8 +560,12 @@ def e2e_leg(wl, host, dev, device, steps, warmup):
         H = torch.zeros((B, wl["K"] - 1, D), device=device)
 
     def step():
-        for k in hx:
+        for k in dx:
             dx[k].copy_(hx[k], non_blocking=True)
+        if streamed:
+            xh = [hx[k].view(torch.bfloat16) for k in ("x1", "x2", "x3")]
+            hy.modal_long_conv_host(*xh, dx["a"], dx["R"], dx["Ds"], y=y_host, workspace=hws)
+            return
         bf = {k: dx[k].view(torch.bfloat16) for k in ("x1", "x2", "x3", "xp") if k in dx}
         if wl.get("cx"):
             hy.modal_long_conv_complex(bf["x1"], bf["x2"], bf["x3"], dx["a"], dx["R"], dx["Ds"], y=y, workspace=ws)
@@ -577,8 +591,10 @@ def e2e_leg(wl, host, dev, device, steps, warmup):
         y_host.copy_(y.view(torch.int16), non_blocking=True)
 
     per = time_steps(step, steps, warmup, device)
-    if wl["kind"] == "modal":
-        hy.workspace_check(ws)  # a launch whose bounded wait gave up is an error, not a timing
+    if streamed:
+        hy.workspace_check(hws)  # a launch whose bounded wait gave up is an error, not a timing
+    elif wl["kind"] == "modal":
+        hy.workspace_check(ws)
     h2d = sum(v.numel() * v.element_size() for v in hx.values())
     d2h = y_host.numel() * y_host.element_size()
     return per, h2d, d2h

@@ -35,6 +35,8 @@ __all__ = [
     "modal_long_conv",
     "modal_long_conv_complex",
     "modal_long_conv_complex_packed",
+    "HostWorkspace",
+    "modal_long_conv_host",
     "modal_long_conv_packed",
     "modal_state_init",
     "short_conv",
@@ -172,6 +174,73 @@ def modal_long_conv(x1, x2, x3, log_poles, residues, Dskip=None, y=None, state_i
                                      _ptr(Dskip), _ptr(y), ld_y, _ptr(state_in), _ptr(state_out),
                                      B, L, D, N, _ptr(workspace.buf), workspace.nbytes, _stream(stream))
     check("hyena_modal_long_conv", rc)
+    return y
+
+
+def _host_bld(x, name):
+    """[B, L, D] bf16 (or int16 bits) host tensor with unit channel stride ->
+    (B, L, D, ld)."""
+    torch = _torch()
+    if x.dtype not in (torch.bfloat16, torch.int16) or x.dim() != 3 or x.is_cuda:
+        raise ValueError(f"{name} must be a 3-D bf16 host tensor [B, L, D]")
+    B, L, D = x.shape
+    if x.stride(2) != 1:
+        raise ValueError(f"{name} must be channel-contiguous")
+    ld = x.stride(1) if L > 1 else (x.stride(0) // max(L, 1) if B > 1 else D)
+    if B > 1 and L > 0 and x.stride(0) != L * ld:
+        raise ValueError(f"{name}: batch stride must equal L * row stride")
+    return B, L, D, ld
+
+
+class HostWorkspace:
+    """Device workspace of modal_long_conv_host (the scan's workspace, two
+    staging slots of `chunk` tokens and the carried state), zero-filled once."""
+
+    def __init__(self, B: int, D: int, N: int, chunk: int = 2048, device=None, stream=None):
+        torch = _torch()
+        n = int(lib().hyena_modal_host_workspace_size(B, D, N, chunk))
+        if n == 0:
+            raise ValueError("invalid host-workspace shape (chunk must be a positive multiple of 128)")
+        self.nbytes, self.chunk = n, chunk
+        self.buf = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+        check("hyena_modal_workspace_init",
+              lib().hyena_modal_workspace_init(_ptr(self.buf), n, _stream(stream)))
+
+
+def modal_long_conv_host(x1, x2, x3, log_poles, residues, Dskip=None, y=None, state_in=None,
+                         state_out=None, workspace: HostWorkspace | None = None, stream=None):
+    """modal_long_conv with x1, x2, x3 and y in host memory ([B, L, D] bf16
+    host tensors, pinned for overlapped copies): the sequence is streamed
+    through the device in chunks of ``workspace.chunk`` tokens with the copies
+    in both directions overlapping the scan.  Parameters and state are device
+    tensors.  Returns y (a host tensor, allocated pinned if not given); it is
+    valid once ``stream`` has been synchronised."""
+    torch = _torch()
+    s1, s2, s3 = _host_bld(x1, "x1"), _host_bld(x2, "x2"), _host_bld(x3, "x3")
+    _same_ld(s1, s2, s3)
+    B, L, D, ld = s1
+    if s2[:3] != (B, L, D) or s3[:3] != (B, L, D):
+        raise ValueError("x1, x2, x3 shapes differ")
+    Dn, N = log_poles.shape
+    if Dn != D:
+        raise ValueError("log_poles must be [D, N]")
+    _f32(log_poles, (D, N), "log_poles", False)
+    _f32(residues, (D, N), "residues", False)
+    _f32(Dskip, (D,), "Dskip")
+    _f32(state_in, (B, D, N), "state_in")
+    _f32(state_out, (B, D, N), "state_out")
+    if y is None:
+        y = torch.empty((B, L, D), dtype=torch.bfloat16).pin_memory()
+    yB, yL, yD, ld_y = _host_bld(y, "y")
+    if (yB, yL, yD) != (B, L, D):
+        raise ValueError("y shape differs from x")
+    if workspace is None:
+        workspace = HostWorkspace(B, D, N, device=log_poles.device, stream=stream)
+    rc = lib().hyena_modal_long_conv_host(_ptr(x1), _ptr(x2), _ptr(x3), ld, _ptr(log_poles), _ptr(residues),
+                                          _ptr(Dskip), _ptr(y), ld_y, _ptr(state_in), _ptr(state_out),
+                                          B, L, D, N, workspace.chunk, _ptr(workspace.buf), workspace.nbytes,
+                                          _stream(stream))
+    check("hyena_modal_long_conv_host", rc)
     return y
 
 

@@ -169,6 +169,7 @@ void record_cuda_error(cudaError_t e, const char *where)
 void record_message(const char *msg) { snprintf(g_last_error, sizeof g_last_error, "%s", msg); }
 
 void add_launches(int n) { g_last_launches += n; }
+void set_last_launches(int n) { g_last_launches = n; }
 
 ModalLayout modal_layout(int B, int D, int N)
 {

@@ -18,6 +18,7 @@ void record_message(const char *msg);
 // Adds to the launch count that hyena_last_launch_count reports for the
 // calling thread's most recent call.
 void add_launches(int n);
+void set_last_launches(int n);  // the launch count hyena_last_launch_count reports
 
 #define HYENA_TRY(call, where)                       \
     do {                                             \

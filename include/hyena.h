@@ -145,6 +145,46 @@ hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t 
                                      void *stream);
 
 /*
+ * hyena_modal_long_conv over inputs and outputs in HOST memory (no
+ * counterpart on the pages: the chunked prefill of the Evo2-7B-262K model
+ * card's "Custom cache" and the turboquant-evo2-int4 card's §"Chunk size",
+ * applied to a sequence that is not resident on the device).
+ *
+ * x1, x2, x3 [B, L, ld_x] and y [B, L, ld_y] are host pointers (bf16); page-
+ * locked memory (cudaHostAlloc / cudaHostRegister) lets the copies overlap,
+ * pageable memory works but serialises them.  log_poles, residues, Dskip,
+ * state_in and state_out are device pointers as in hyena_modal_long_conv.
+ * The sequence is streamed through the device in chunks of `chunk` tokens
+ * (a positive multiple of 128): while chunk i is scanned on `stream`, chunk
+ * i+1 is copied host->device and chunk i-1's output device->host on two copy
+ * streams the library owns (one pair per device), so the host link carries
+ * both directions at once.  The modal state is carried from chunk to chunk,
+ * and because every chunk boundary is a unit boundary y and state_out equal
+ * the single pass bit for bit.
+ * workspace  device, >= hyena_modal_host_workspace_size(B, D, N, chunk)
+ *            bytes, 256-byte aligned, zero-filled once by
+ *            hyena_modal_workspace_init: the scan's workspace, two staging
+ *            slots of x1/x2/x3/y for `chunk` tokens and the carried state.
+ * On return the work is enqueued; `stream` is ordered after the last copy to
+ * the host, so synchronising `stream` makes y valid.  Not capturable into a
+ * CUDA graph (it orders the library's copy streams with events); calls on
+ * one device are enqueued one at a time (a lock), and calls sharing a
+ * workspace must not overlap in time.  Errors as hyena_modal_long_conv, plus
+ * HYENA_ERR_INVALID_ARG for a chunk that is not a positive multiple of 128.
+ */
+size_t hyena_modal_host_workspace_size(int B, int D, int N, int chunk);
+
+hyena_status_t hyena_modal_long_conv_host(const hyena_bf16_t *x1, const hyena_bf16_t *x2,
+                                          const hyena_bf16_t *x3, int64_t ld_x,
+                                          const float *log_poles, const float *residues,
+                                          const float *Dskip,
+                                          hyena_bf16_t *y, int64_t ld_y,
+                                          const float *state_in, float *state_out,
+                                          int B, int L, int D, int N, int chunk,
+                                          void *workspace, size_t workspace_bytes,
+                                          void *stream);
+
+/*
  * Allocation-free variant of hyena_modal_long_conv (no counterpart on the
  * pages: it exists for callers of this library that must not allocate device
  * memory).  Some callers cannot call cudaMalloc or take memory from an

@@ -205,6 +205,33 @@ def test_other_entry_points_reject_bad_arguments():
     assert lib.hyena_workspace_check(None, None) == INVALID
 
 
+def test_host_buffer_entry_point_sizes_and_bad_arguments():
+    lib = hy.lib()
+    ws = lib.hyena_modal_host_workspace_size
+    assert ws(1, 4096, 16, 100) == 0  # not a multiple of 128
+    assert ws(1, 4096, 16, 0) == 0
+    assert ws(1, 4096, 16, 2048) > 0
+    assert ws(1, 4096, hy.MAX_MODES + 1, 2048) == 0
+    # two staging slots of x1, x2, x3, y (8 bytes per channel-token each) on
+    # top of the scan's workspace and the carried state
+    extra = ws(1, 4096, 16, 2048) - lib.hyena_modal_long_conv_workspace_size(1, 4096, 16)
+    assert extra >= 2 * 2048 * 4096 * 8 + 4096 * 16 * 4
+
+    def conv(x=A, L=256, D=64, N=8, chunk=128, w=A, wb=1 << 30, ld_x=None, ld_y=None):
+        return lib.hyena_modal_long_conv_host(x, x, x, ld_x or D, A, A, None, x, ld_y or D, None, None,
+                                              1, L, D, N, chunk, w, wb, None)
+    assert conv(chunk=100) == INVALID
+    assert conv(chunk=0) == INVALID
+    assert conv(x=None) == INVALID
+    assert conv(N=0) == INVALID
+    assert conv(N=hy.MAX_MODES + 1) == UNSUP
+    assert conv(ld_x=32) == INVALID
+    assert conv(D=60) == ALIGN
+    assert conv(w=None) == WORKSPACE
+    assert conv(wb=1024) == WORKSPACE
+    assert conv(w=A + 16) == ALIGN
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "SO", str(tmp_path / "missing.so"))
     monkeypatch.setattr(_lib, "_lib", None)

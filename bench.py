@@ -541,17 +541,20 @@ def e2e_leg(wl, host, dev, device, steps, warmup):
         return t.pin_memory()
 
     hx = {k: pin(v) for k, v in host.items()}
-    # The real-mode prefill streams its host buffers through the library's
-    # host-buffer entry point (chunks of whole units, copies in both
-    # directions overlapping the scan); everything else copies them here.
-    streamed = wl["kind"] == "modal" and not (wl.get("cx") or wl.get("group") or wl.get("decode"))
+    # Prefill with separate inputs (real modes, FIR) streams its host buffers
+    # through the library's host-buffer entry points (chunks, copies in both
+    # directions overlapping the computation); everything else copies here.
+    streamed = not (wl.get("cx") or wl.get("group") or wl.get("decode"))
     on_host = ("x1", "x2", "x3") if streamed else ()
     dx = {k: torch.empty(v.shape, dtype=v.dtype, device=device) for k, v in hx.items() if k not in on_host}
     y_host = torch.empty((wl["B"], wl["L"], wl["D"]), dtype=torch.int16).pin_memory()
     B, L, D = wl["B"], wl["L"], wl["D"]
     y = torch.empty((B, L, D), dtype=torch.bfloat16, device=device)
-    if streamed:
+    if streamed and wl["kind"] == "modal":
         hws = hy.HostWorkspace(B, D, wl["N"], chunk=E2E_CHUNK, device=device)
+    elif streamed:
+        hws_fir = torch.empty(int(hy.lib().hyena_short_host_workspace_size(B, D, wl["K"], E2E_CHUNK)),
+                              dtype=torch.uint8, device=device)
     if wl["kind"] == "modal":
         cx = bool(wl.get("cx"))
         ws = hy.ModalWorkspace(B, D, (2 if cx else 1) * wl["N"], device=device)
@@ -564,7 +567,11 @@ def e2e_leg(wl, host, dev, device, steps, warmup):
             dx[k].copy_(hx[k], non_blocking=True)
         if streamed:
             xh = [hx[k].view(torch.bfloat16) for k in ("x1", "x2", "x3")]
-            hy.modal_long_conv_host(*xh, dx["a"], dx["R"], dx["Ds"], y=y_host, workspace=hws)
+            if wl["kind"] == "modal":
+                hy.modal_long_conv_host(*xh, dx["a"], dx["R"], dx["Ds"], y=y_host, workspace=hws)
+            else:
+                hy.short_conv_host(*xh, dx["taps"].view(torch.bfloat16), None, y=y_host, chunk=E2E_CHUNK,
+                                   workspace=hws_fir)
             return
         bf = {k: dx[k].view(torch.bfloat16) for k in ("x1", "x2", "x3", "xp") if k in dx}
         if wl.get("cx"):
@@ -591,7 +598,7 @@ def e2e_leg(wl, host, dev, device, steps, warmup):
         y_host.copy_(y.view(torch.int16), non_blocking=True)
 
     per = time_steps(step, steps, warmup, device)
-    if streamed:
+    if streamed and wl["kind"] == "modal":
         hy.workspace_check(hws)  # a launch whose bounded wait gave up is an error, not a timing
     elif wl["kind"] == "modal":
         hy.workspace_check(ws)

@@ -37,6 +37,7 @@ __all__ = [
     "modal_long_conv_complex_packed",
     "HostWorkspace",
     "modal_long_conv_host",
+    "short_conv_host",
     "modal_long_conv_packed",
     "modal_state_init",
     "short_conv",
@@ -241,6 +242,43 @@ def modal_long_conv_host(x1, x2, x3, log_poles, residues, Dskip=None, y=None, st
                                           B, L, D, N, workspace.chunk, _ptr(workspace.buf), workspace.nbytes,
                                           _stream(stream))
     check("hyena_modal_long_conv_host", rc)
+    return y
+
+
+def short_conv_host(x1, x2, x3, taps, Dskip=None, y=None, hist_in=None, hist_out=None, chunk=2048,
+                    workspace=None, stream=None):
+    """short_conv with x1, x2, x3 and y in host memory ([B, L, D] bf16 host
+    tensors, pinned for overlapped copies), streamed through the device in
+    chunks with the FIR window carried.  taps [D, K] bf16, Dskip, hist_in and
+    hist_out ([B, K-1, D] fp32) are device tensors; ``workspace`` is a device
+    uint8 tensor of at least short_host_workspace_size bytes (allocated if
+    not given).  Returns y, valid once ``stream`` has been synchronised."""
+    torch = _torch()
+    s1, s2, s3 = _host_bld(x1, "x1"), _host_bld(x2, "x2"), _host_bld(x3, "x3")
+    _same_ld(s1, s2, s3)
+    B, L, D, ld = s1
+    if s2[:3] != (B, L, D) or s3[:3] != (B, L, D):
+        raise ValueError("x1, x2, x3 shapes differ")
+    if taps.dtype != torch.bfloat16 or taps.dim() != 2 or taps.shape[0] != D or not taps.is_contiguous():
+        raise ValueError("taps must be a contiguous [D, K] bf16 tensor")
+    K = taps.shape[1]
+    _f32(Dskip, (D,), "Dskip")
+    _f32(hist_in, (B, K - 1, D), "hist_in")
+    _f32(hist_out, (B, K - 1, D), "hist_out")
+    if y is None:
+        y = torch.empty((B, L, D), dtype=torch.bfloat16).pin_memory()
+    yB, yL, yD, ld_y = _host_bld(y, "y")
+    if (yB, yL, yD) != (B, L, D):
+        raise ValueError("y shape differs from x")
+    need = int(lib().hyena_short_host_workspace_size(B, D, K, chunk))
+    if need == 0:
+        raise ValueError("invalid host-workspace shape")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=taps.device)
+    rc = lib().hyena_short_conv_host(_ptr(x1), _ptr(x2), _ptr(x3), ld, _ptr(taps), _ptr(Dskip), _ptr(y), ld_y,
+                                     _ptr(hist_in), _ptr(hist_out), B, L, D, K, chunk, _ptr(workspace),
+                                     workspace.numel(), _stream(stream))
+    check("hyena_short_conv_host", rc)
     return y
 
 

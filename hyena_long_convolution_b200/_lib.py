@@ -42,6 +42,8 @@ SIGNATURES = {
     "hyena_modal_host_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "hyena_modal_long_conv_host": (_I, [_P, _P, _P, _I64, _P, _P, _P, _P, _I64, _P, _P,
                                         _I, _I, _I, _I, _I, _P, _SZ, _P]),
+    "hyena_short_host_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "hyena_short_conv_host": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I64, _P, _P, _I, _I, _I, _I, _I, _P, _SZ, _P]),
     "hyena_modal_noalloc_check": (_I, [_P]),
     "hyena_modal_noalloc_scratch": (_I, [_P, _P]),
     "hyena_modal_decode": (_I, [_P, _P, _P, _I64, _P, _P, _P, _P, _I64, _P, _I, _I, _I, _P]),

@@ -185,6 +185,28 @@ hyena_status_t hyena_modal_long_conv_host(const hyena_bf16_t *x1, const hyena_bf
                                           void *stream);
 
 /*
+ * hyena_short_conv over inputs and outputs in HOST memory, streamed like
+ * hyena_modal_long_conv_host with the FIR window carried from chunk to chunk
+ * (Evo1-1.5-7B-8K model card, "Cache subclass": the FIR window).  Any chunk
+ * >= 1 gives y and hist_out equal to the single pass bit for bit.  taps,
+ * Dskip, hist_in and hist_out are device pointers as in hyena_short_conv.
+ * workspace  device, >= hyena_short_host_workspace_size(B, D, K, chunk)
+ *            bytes, 256-byte aligned (no initialisation needed): two staging
+ *            slots of x1/x2/x3/y for `chunk` tokens and the carried window.
+ * Ordering, locking and graph capture as hyena_modal_long_conv_host.
+ */
+size_t hyena_short_host_workspace_size(int B, int D, int K, int chunk);
+
+hyena_status_t hyena_short_conv_host(const hyena_bf16_t *x1, const hyena_bf16_t *x2,
+                                     const hyena_bf16_t *x3, int64_t ld_x,
+                                     const hyena_bf16_t *taps, const float *Dskip,
+                                     hyena_bf16_t *y, int64_t ld_y,
+                                     const float *hist_in, float *hist_out,
+                                     int B, int L, int D, int K, int chunk,
+                                     void *workspace, size_t workspace_bytes,
+                                     void *stream);
+
+/*
  * Allocation-free variant of hyena_modal_long_conv (no counterpart on the
  * pages: it exists for callers of this library that must not allocate device
  * memory).  Some callers cannot call cudaMalloc or take memory from an

@@ -232,6 +232,26 @@ def test_host_buffer_entry_point_sizes_and_bad_arguments():
     assert conv(w=A + 16) == ALIGN
 
 
+def test_short_host_buffer_entry_point_sizes_and_bad_arguments():
+    lib = hy.lib()
+    ws = lib.hyena_short_host_workspace_size
+    assert ws(1, 4096, 128, 0) == 0
+    assert ws(1, 4096, 129, 2048) == 0
+    assert ws(2, 4096, 128, 2048) >= 2 * 4 * 2 * 2048 * 4096 * 2 + 2 * 127 * 4096 * 4
+
+    def conv(x=A, L=256, D=64, K=7, chunk=128, w=A, wb=1 << 30, ld_x=None):
+        return lib.hyena_short_conv_host(x, x, x, ld_x or D, A, None, x, D, None, None, 1, L, D, K, chunk, w, wb, None)
+    assert conv(chunk=0) == INVALID
+    assert conv(x=None) == INVALID
+    assert conv(K=0) == INVALID
+    assert conv(K=129) == UNSUP
+    assert conv(ld_x=32) == INVALID
+    assert conv(D=60) == ALIGN
+    assert conv(w=None) == WORKSPACE
+    assert conv(wb=1024) == WORKSPACE
+    assert conv(w=A + 16) == ALIGN
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "SO", str(tmp_path / "missing.so"))
     monkeypatch.setattr(_lib, "_lib", None)

@@ -1,11 +1,13 @@
-"""The host-buffer modal conv (hyena_modal_long_conv_host).
+"""The host-buffer entry points (hyena_modal_long_conv_host,
+hyena_short_conv_host).
 
 Inputs and outputs live in page-locked host memory and are streamed through
-the device in chunks of whole 128-token units with the state carried, so y
-and the final state must equal the device-resident single pass bit for bit,
+the device in chunks (whole 128-token units for the modal filter, any length
+for the FIR) with the state or window carried, so y and the final state must
+equal the device-resident single pass bit for bit,
 for ragged sequence lengths, several batch rows, padded host rows, a carried
-input state and every chunk size; and stay within tolerance of the fp64
-oracle.
+input state or window and every chunk size; and stay within tolerance of the
+fp64 oracle.
 """
 import numpy as np
 import pytest
@@ -73,3 +75,32 @@ def test_host_stream_against_the_oracle():
     assert_close(y, ref_y, "host-buffer modal conv")
     rel, _ = metrics(S_host.cpu().numpy().astype(np.float64), ref_S)
     assert rel < 1e-4
+
+
+@pytest.mark.parametrize("B,L,D,K,chunk", [
+    (2, 3000, 136, 7, 1000),     # hcs, chunks not a multiple of anything
+    (1, 5000, 256, 128, 777),    # hcm, chunks longer than the window, ragged
+    (1, 300, 64, 128, 64),       # every chunk shorter than the window
+])
+def test_short_host_stream_is_bitwise_the_device_single_pass(B, L, D, K, chunk):
+    import torch
+    import hyena_long_convolution_b200 as hy
+    from synth import make_fir_inputs
+    inp = make_fir_inputs(B, L, D, K, seed=L + K, with_skip=True)
+    taps = to_dev_bf16(inp["taps"])
+    Ds = to_dev_f32(inp["Dskip"])
+    H0 = np.random.default_rng(K).standard_normal((B, K - 1, D)).astype(np.float32)
+    H_in = torch.from_numpy(H0).cuda()
+    xd = [to_dev_bf16(inp[k]) for k in ("x1", "x2", "x3")]
+    H_dev = torch.empty_like(H_in)
+    y_dev = hy.short_conv(*xd, taps, Ds, hist_in=H_in, hist_out=H_dev)
+    xh = [_host_bf16(inp[k]) for k in ("x1", "x2", "x3")]
+    yh = _host_bf16(np.zeros((B, L, D), np.uint16))
+    H_host = torch.empty_like(H_in)
+    hy.short_conv_host(*xh, taps, Ds, y=yh, hist_in=H_in, hist_out=H_host, chunk=chunk)
+    torch.cuda.synchronize()
+    assert torch.equal(yh.contiguous().view(torch.int16), y_dev.view(torch.int16).cpu())
+    assert torch.equal(H_host, H_dev)
+    if K == 128 and L == 5000:
+        ref_y, ref_H = oracle.fir(inp["x1"], inp["x2"], inp["x3"], inp["taps"], inp["Dskip"], H0.astype(np.float64))
+        assert_close(from_dev_bf16(yh.contiguous().view(torch.bfloat16)), ref_y, "host-buffer short conv")

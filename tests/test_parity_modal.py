@@ -167,3 +167,17 @@ def test_many_modes_whole_unit_chunks_are_bit_exact(N):
     yc, sc = check(inp, S0, chunks=[256, 128, 640])
     assert np.array_equal(bits_of(yc), bits_of(y1))
     assert np.array_equal(sc.cpu().numpy(), s1.cpu().numpy())
+
+
+@pytest.mark.parametrize("chunks", [[1024] * 6, [3072, 3072], [4096, 2048], [128, 5888, 128]])
+def test_short_and_lookback_paths_agree_bitwise(chunks):
+    # The single pass (48 units per chain) runs the look-back kernel; chunks of
+    # at most 24 units run the two-pass short-sequence path, longer ones the
+    # look-back kernel again.  Both form every value by the same operations,
+    # so any mix of them reproduces the single pass bit for bit.
+    inp = make_modal_inputs(1, 6144, 520, 12, seed=31)
+    S0 = np.random.default_rng(31).standard_normal((1, 520, 12))
+    y1, s1 = check(inp, S0)
+    yc, sc = run_gpu(inp, S0, chunks=chunks)
+    assert np.array_equal(bits_of(yc), bits_of(y1))
+    assert np.array_equal(sc.cpu().numpy(), s1.cpu().numpy())

@@ -507,6 +507,42 @@ __global__ void __launch_bounds__(FW * 32, 4)
 // hist_out[b][j][c] = v[L-H+j] (from hist_in when that index is negative).
 // One thread per (batch row, channel pair) walks j upward, so reading
 // hist_in[j + L] before writing hist_out[j + L] keeps in-place use safe.
+// hist_out row j = v[L - H + j]: from x (t >= 0), from hist_in (t < 0), or
+// zero.  One thread per (batch row, history row, channel pair): every output
+// element is independent, so the launch is as wide as the history.  Used
+// unless hist_out aliases hist_in and 0 < L < H (then rows move within the
+// buffer and the ordered kernel below runs instead).
+__global__ void fir_history_rows_kernel(const FirArgs A)
+{
+    const int pairs = A.D / 2;
+    const int H = A.K - 1;
+    const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= static_cast<long long>(A.B) * H * pairs) return;
+    const int b = static_cast<int>(idx / (static_cast<long long>(H) * pairs));
+    const int rem = static_cast<int>(idx - static_cast<long long>(b) * H * pairs);
+    const int j = rem / pairs;
+    const int c = (rem - j * pairs) * 2;
+    const int t = A.L - H + j;
+    float2 v;
+    if (t >= 0) {
+        const size_t row = (static_cast<size_t>(b) * A.L + t) * A.ld_x;
+        const size_t i0 = row + x_col(c, A.group), i1 = row + x_col(c + 1, A.group);
+        const float2 x1 = make_float2(__uint_as_float(static_cast<uint32_t>(A.x1[i0]) << 16),
+                                      __uint_as_float(static_cast<uint32_t>(A.x1[i1]) << 16));
+        const float2 x2 = make_float2(__uint_as_float(static_cast<uint32_t>(A.x2[i0]) << 16),
+                                      __uint_as_float(static_cast<uint32_t>(A.x2[i1]) << 16));
+        v = __fmul2_rn(x1, x2);
+    } else if (A.hist_in != nullptr) {
+        v = *reinterpret_cast<const float2 *>(A.hist_in + (static_cast<size_t>(b) * H + (H + t)) * A.D + c);
+    } else {
+        v = make_float2(0.f, 0.f);
+    }
+    *reinterpret_cast<float2 *>(A.hist_out + (static_cast<size_t>(b) * H + j) * A.D + c) = v;
+}
+
+// The same values, one thread per (batch row, channel pair) walking the rows
+// forward: hist_out row j is written only after row L + j, its source in the
+// aliased buffer, has been read.
 __global__ void fir_history_kernel(const FirArgs A)
 {
     const int pairs = A.D / 2;
@@ -584,8 +620,14 @@ int launch_fir(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &
         ++launches;
     }
     if (a.hist_out != nullptr && a.K > 1) {
-        const int threads = a.B * (a.D / 2);
-        fir_history_kernel<<<(threads + 255) / 256, 256, 0, st>>>(a);
+        const int H = a.K - 1;
+        if (a.hist_in == a.hist_out && a.L > 0 && a.L < H) {
+            const int threads = a.B * (a.D / 2);
+            fir_history_kernel<<<(threads + 255) / 256, 256, 0, st>>>(a);
+        } else {
+            const long long threads = static_cast<long long>(a.B) * H * (a.D / 2);
+            fir_history_rows_kernel<<<static_cast<unsigned int>((threads + 255) / 256), 256, 0, st>>>(a);
+        }
         HYENA_TRY(cudaGetLastError(), "fir history launch");
         ++launches;
     }

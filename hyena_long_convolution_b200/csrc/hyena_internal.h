@@ -110,10 +110,11 @@ struct ModalSynthArgs {
     float *coef;
 };
 
-// Up to 16 mode slots (the common case) the scan runs as the two-CTAs-per-SM
-// kernel of modal_scan.cu: each compute warp sweeps its unit's aggregate and
-// then its outputs, streaming chunks of MCK rows x MCH channels of x1/x2 (and
-// x3).  With 32 or 64 slots it runs as the warp-specialised kernel of
+// Up to 16 mode slots (the common case) the scan runs as the look-back kernel
+// of modal_scan.cu (two or three CTAs per SM): each compute warp sweeps its
+// unit's aggregate and then its outputs, streaming chunks of MCK rows x MCH
+// channels of x1/x2 (and x3); short sequences take that file's two-pass path
+// (below).  With 32 or 64 slots the scan runs as the warp-specialised kernel of
 // modal_scan_wide.cu (chains of MCH / LPC channels; aggregate warps read
 // chunks of MA_ROWS rows, output warps chunks of MC_ROWS rows).
 constexpr int MCK = 16;
@@ -142,6 +143,7 @@ int launch_modal_narrow(const CUtensorMap &m1, const CUtensorMap &m2, const CUte
 struct ModalMaps {
     CUtensorMap a1, a2, c1, c2, c3, coef;
 };
+
 // Short sequences: up to 16 slots, at most MSHORT_UNITS units per chain whose
 // x1/x2 rows (B L D 4 bytes, 6 for triples) fit in MSHORT_L2_BYTES of L2.
 // There the scan runs as two plain passes over all units at once (aggregates,

@@ -261,7 +261,10 @@ class ClockSampler:
                 ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
             except ValueError:
                 ts = None
-            if ts is not None and t0 is not None and t1 is not None and not (t0 - 0.05 <= ts <= t1 + 0.05):
+            # a short timed region can fall between two 50 ms samples: then the
+            # samples within 0.3 s of it stand in (counted in "samples")
+            slack = 0.05 if t0 is None or t1 is None or t1 - t0 > 0.5 else 0.3
+            if ts is not None and t0 is not None and t1 is not None and not (t0 - slack <= ts <= t1 + slack):
                 continue
             try:
                 sm.append(float(parts[2]))

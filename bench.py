@@ -482,13 +482,17 @@ class Step:
             return
         if wl["kind"] == "modal":
             if wl.get("chunk"):
+                # chunked prefill of one sequence: the filter is synthesised
+                # once, then every chunk runs with the carried state
                 hy.modal_state_init(self.S)
+                n += hy.last_launch_count()
+                hy.modal_prepare(d["a"], d["R"], d["Ds"], self.ws, B=wl["B"])
                 n += hy.last_launch_count()
                 c = wl["chunk"]
                 for t0 in range(0, wl["L"], c):
                     sl = slice(t0, t0 + c)
-                    hy.modal_long_conv(d["x1"][:, sl], d["x2"][:, sl], d["x3"][:, sl], d["a"], d["R"], d["Ds"],
-                                       y=self.y[:, sl], state_in=self.S, state_out=self.S, workspace=self.ws)
+                    hy.modal_long_conv_prepared(d["x1"][:, sl], d["x2"][:, sl], d["x3"][:, sl], wl["N"], self.ws,
+                                                y=self.y[:, sl], state_in=self.S, state_out=self.S)
                     n += hy.last_launch_count()
             else:
                 hy.modal_long_conv(d["x1"], d["x2"], d["x3"], d["a"], d["R"], d["Ds"], y=self.y,

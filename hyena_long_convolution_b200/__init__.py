@@ -37,6 +37,8 @@ __all__ = [
     "modal_long_conv_complex_packed",
     "HostWorkspace",
     "modal_long_conv_host",
+    "modal_prepare",
+    "modal_long_conv_prepared",
     "short_conv_host",
     "modal_long_conv_packed",
     "modal_state_init",
@@ -175,6 +177,42 @@ def modal_long_conv(x1, x2, x3, log_poles, residues, Dskip=None, y=None, state_i
                                      _ptr(Dskip), _ptr(y), ld_y, _ptr(state_in), _ptr(state_out),
                                      B, L, D, N, _ptr(workspace.buf), workspace.nbytes, _stream(stream))
     check("hyena_modal_long_conv", rc)
+    return y
+
+
+def modal_prepare(log_poles, residues, Dskip, workspace: ModalWorkspace, B: int = 1, stream=None):
+    """Form the coefficient table of a real-mode filter in ``workspace`` once,
+    for the chunks of one sequence that follow (modal_long_conv_prepared)."""
+    D, N = log_poles.shape
+    _f32(log_poles, (D, N), "log_poles", False)
+    _f32(residues, (D, N), "residues", False)
+    _f32(Dskip, (D,), "Dskip")
+    rc = lib().hyena_modal_prepare(_ptr(log_poles), _ptr(residues), _ptr(Dskip), B, D, N, _ptr(workspace.buf),
+                                   workspace.nbytes, _stream(stream))
+    check("hyena_modal_prepare", rc)
+
+
+def modal_long_conv_prepared(x1, x2, x3, N: int, workspace: ModalWorkspace, y=None, state_in=None, state_out=None,
+                             stream=None):
+    """modal_long_conv with the table of the last modal_prepare on ``workspace``
+    (the same bits as modal_long_conv with those parameters)."""
+    torch = _torch()
+    s1, s2, s3 = _bld(x1, "x1"), _bld(x2, "x2"), _bld(x3, "x3")
+    _same_ld(s1, s2, s3)
+    B, L, D, ld = s1
+    if s2[:3] != (B, L, D) or s3[:3] != (B, L, D):
+        raise ValueError("x1, x2, x3 shapes differ")
+    _f32(state_in, (B, D, N), "state_in")
+    _f32(state_out, (B, D, N), "state_out")
+    if y is None:
+        y = torch.empty((B, L, D), dtype=torch.bfloat16, device=x1.device)
+    yB, yL, yD, ld_y = _bld(y, "y")
+    if (yB, yL, yD) != (B, L, D):
+        raise ValueError("y shape differs from x")
+    rc = lib().hyena_modal_long_conv_prepared(_ptr(x1), _ptr(x2), _ptr(x3), ld, _ptr(y), ld_y, _ptr(state_in),
+                                              _ptr(state_out), B, L, D, N, _ptr(workspace.buf), workspace.nbytes,
+                                              _stream(stream))
+    check("hyena_modal_long_conv_prepared", rc)
     return y
 
 

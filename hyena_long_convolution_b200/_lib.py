@@ -39,6 +39,8 @@ SIGNATURES = {
                                    _I, _I, _I, _I, _P, _SZ, _P]),
     "hyena_modal_long_conv_noalloc": (_I, [_P, _P, _P, _I64, _P, _P, _P, _P, _I64, _P, _P,
                                            _I, _I, _I, _I, _P]),
+    "hyena_modal_prepare": (_I, [_P, _P, _P, _I, _I, _I, _P, _SZ, _P]),
+    "hyena_modal_long_conv_prepared": (_I, [_P, _P, _P, _I64, _P, _I64, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
     "hyena_modal_host_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "hyena_modal_long_conv_host": (_I, [_P, _P, _P, _I64, _P, _P, _P, _P, _I64, _P, _P,
                                         _I, _I, _I, _I, _I, _P, _SZ, _P]),

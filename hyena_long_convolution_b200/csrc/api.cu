@@ -262,16 +262,18 @@ hyena_status_t short_conv_impl(const XSource &xs, const hyena_bf16_t *taps, cons
 
 // cx: complex modes; the N of the caller counts modes, the kernels count
 // slots (two per complex mode).
+// With `synth` false the coefficient table is the one hyena_modal_prepare left
+// in the workspace and the filter parameters are not used.
 hyena_status_t modal_long_conv_impl(const XSource &xs, const float *log_poles, const float *residues,
                                    const float *Dskip, hyena_bf16_t *y, int64_t ld_y, const float *state_in,
                                    float *state_out, int B, int L, int D, int N, void *workspace,
-                                   size_t workspace_bytes, void *stream, bool cx = false)
+                                   size_t workspace_bytes, void *stream, bool cx = false, bool synth = true)
 {
     hyena_status_t st = HYENA_OK;
     if (N < 1) return HYENA_ERR_INVALID_ARG;
     if (N > (cx ? HYENA_MAX_COMPLEX_MODES : HYENA_MAX_MODES)) return HYENA_ERR_UNSUPPORTED;
     if (cx) N *= 2;
-    if (!log_poles || !residues) return HYENA_ERR_INVALID_ARG;
+    if (synth && (!log_poles || !residues)) return HYENA_ERR_INVALID_ARG;
     if (!aligned16(log_poles) || !aligned16(residues) || (Dskip && !aligned16(Dskip)) ||
         (state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
         return HYENA_ERR_ALIGNMENT;
@@ -321,7 +323,7 @@ hyena_status_t modal_long_conv_impl(const XSource &xs, const float *log_poles, c
     sy.Dp = lay.Dp;
     sy.coef = reinterpret_cast<float *>(ws + lay.off_coef);
 
-    const int ns = launch_modal_synth(sy, lay.NP, cx, s);
+    const int ns = synth ? launch_modal_synth(sy, lay.NP, cx, s) : 0;
     if (ns < 0) return HYENA_ERR_CUDA;
     int n = -1;
     if (lay.LPC == 1) {
@@ -484,6 +486,42 @@ hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t 
     if (st != HYENA_OK) return st;
     return modal_long_conv_impl(separate_source(x1, x2, x3, ld_x, D), log_poles, residues, Dskip, y, ld_y, state_in,
                                 state_out, B, L, D, N, workspace, workspace_bytes, stream);
+}
+
+hyena_status_t hyena_modal_prepare(const float *log_poles, const float *residues, const float *Dskip, int B, int D,
+                                   int N, void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (B < 1 || D < 1 || N < 1) return HYENA_ERR_INVALID_ARG;
+    if (N > HYENA_MAX_MODES) return HYENA_ERR_UNSUPPORTED;
+    if (!log_poles || !residues) return HYENA_ERR_INVALID_ARG;
+    if (D % 8) return HYENA_ERR_ALIGNMENT;
+    if (!aligned16(log_poles) || !aligned16(residues) || (Dskip && !aligned16(Dskip))) return HYENA_ERR_ALIGNMENT;
+    const ModalLayout lay = modal_layout(B, D, N);
+    if (workspace == nullptr || workspace_bytes < lay.total) return HYENA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return HYENA_ERR_ALIGNMENT;
+    ModalSynthArgs sy{};
+    sy.log_poles = log_poles;
+    sy.residues = residues;
+    sy.Dskip = Dskip;
+    sy.D = D;
+    sy.N = N;
+    sy.Dp = lay.Dp;
+    sy.coef = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + lay.off_coef);
+    const int n = launch_modal_synth(sy, lay.NP, false, static_cast<cudaStream_t>(stream));
+    if (n < 0) return HYENA_ERR_CUDA;
+    g_last_launches = n;
+    return HYENA_OK;
+}
+
+hyena_status_t hyena_modal_long_conv_prepared(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
+                                              int64_t ld_x, hyena_bf16_t *y, int64_t ld_y, const float *state_in,
+                                              float *state_out, int B, int L, int D, int N, void *workspace,
+                                              size_t workspace_bytes, void *stream)
+{
+    const hyena_status_t st = check_x(x1, x2, x3, ld_x, y, ld_y, B, L, D);
+    if (st != HYENA_OK) return st;
+    return modal_long_conv_impl(separate_source(x1, x2, x3, ld_x, D), nullptr, nullptr, nullptr, y, ld_y, state_in,
+                                state_out, B, L, D, N, workspace, workspace_bytes, stream, false, false);
 }
 
 hyena_status_t hyena_modal_long_conv_packed(const hyena_bf16_t *xp, int64_t ld_x, int group, const float *log_poles,

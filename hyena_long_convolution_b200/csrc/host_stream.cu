@@ -194,9 +194,13 @@ extern "C" hyena_status_t hyena_modal_long_conv_host(const hyena_bf16_t *x1, con
                          "host-buffer modal conv",
                          [&](int i, bool last, const hyena_bf16_t *c1, const hyena_bf16_t *c2, const hyena_bf16_t *c3,
                              hyena_bf16_t *cy, int rows) {
-                             return hyena_modal_long_conv(c1, c2, c3, D, log_poles, residues, Dskip, cy, D,
-                                                          i == 0 ? state_in : carry, last ? state_out : carry, B,
-                                                          rows, D, N, modal_ws, lay.modal, stream);
+                             // the first chunk synthesises the filter, the others reuse its table
+                             if (i == 0)
+                                 return hyena_modal_long_conv(c1, c2, c3, D, log_poles, residues, Dskip, cy, D,
+                                                              state_in, last ? state_out : carry, B, rows, D, N,
+                                                              modal_ws, lay.modal, stream);
+                             return hyena_modal_long_conv_prepared(c1, c2, c3, D, cy, D, carry, last ? state_out : carry,
+                                                                   B, rows, D, N, modal_ws, lay.modal, stream);
                          });
 }
 

@@ -145,6 +145,34 @@ hyena_status_t hyena_modal_long_conv(const hyena_bf16_t *x1, const hyena_bf16_t 
                                      void *stream);
 
 /*
+ * Chunked prefill with the filter synthesised once (turboquant-evo2-int4
+ * model card, §"Chunk size": a long prompt is fed in chunks through the same
+ * layer; the filter is the same for every chunk).
+ *
+ * hyena_modal_prepare forms the coefficient table of the real-mode filter
+ * (p = exp(a) with CUDA's expf, residues, skip, p^64, p^128) in `workspace`,
+ * as the first step of every hyena_modal_long_conv call does; arguments and
+ * errors as there (the workspace sized for B, D, N).
+ * hyena_modal_long_conv_prepared is hyena_modal_long_conv without that step:
+ * it uses the table the last hyena_modal_prepare on this workspace left, and
+ * gives the same bits as hyena_modal_long_conv with those parameters.  Any
+ * other modal call on the workspace (hyena_modal_long_conv and its variants)
+ * replaces the table with its own parameters' table; prepare again after it.
+ * Real modes only (complex modes: hyena_modal_long_conv_complex).
+ */
+hyena_status_t hyena_modal_prepare(const float *log_poles, const float *residues, const float *Dskip,
+                                   int B, int D, int N, void *workspace, size_t workspace_bytes,
+                                   void *stream);
+
+hyena_status_t hyena_modal_long_conv_prepared(const hyena_bf16_t *x1, const hyena_bf16_t *x2,
+                                              const hyena_bf16_t *x3, int64_t ld_x,
+                                              hyena_bf16_t *y, int64_t ld_y,
+                                              const float *state_in, float *state_out,
+                                              int B, int L, int D, int N,
+                                              void *workspace, size_t workspace_bytes,
+                                              void *stream);
+
+/*
  * hyena_modal_long_conv over inputs and outputs in HOST memory (no
  * counterpart on the pages: the chunked prefill of the Evo2-7B-262K model
  * card's "Custom cache" and the turboquant-evo2-int4 card's §"Chunk size",

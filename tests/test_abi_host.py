@@ -232,6 +232,30 @@ def test_host_buffer_entry_point_sizes_and_bad_arguments():
     assert conv(w=A + 16) == ALIGN
 
 
+def test_prepared_entry_points_reject_bad_arguments():
+    lib = hy.lib()
+    big = 1 << 30
+
+    def prep(a=A, r=A, D=64, N=8, w=A, wb=big):
+        return lib.hyena_modal_prepare(a, r, None, 1, D, N, w, wb, None)
+    assert prep(a=None) == INVALID
+    assert prep(r=None) == INVALID
+    assert prep(N=0) == INVALID
+    assert prep(N=hy.MAX_MODES + 1) == UNSUP
+    assert prep(D=60) == ALIGN
+    assert prep(a=A + 4) == ALIGN
+    assert prep(w=None) == WORKSPACE
+    assert prep(wb=64) == WORKSPACE
+
+    def conv(x=A, L=256, N=8, w=A, wb=big):
+        return lib.hyena_modal_long_conv_prepared(x, x, x, 64, x, 64, None, None, 1, L, 64, N, w, wb, None)
+    assert conv(x=None) == INVALID
+    assert conv(N=0) == INVALID
+    assert conv(N=hy.MAX_MODES + 1) == UNSUP
+    assert conv(w=None) == WORKSPACE
+    assert conv(wb=64) == WORKSPACE
+
+
 def test_short_host_buffer_entry_point_sizes_and_bad_arguments():
     lib = hy.lib()
     ws = lib.hyena_short_host_workspace_size

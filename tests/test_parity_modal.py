@@ -181,3 +181,28 @@ def test_short_and_lookback_paths_agree_bitwise(chunks):
     yc, sc = run_gpu(inp, S0, chunks=chunks)
     assert np.array_equal(bits_of(yc), bits_of(y1))
     assert np.array_equal(sc.cpu().numpy(), s1.cpu().numpy())
+
+
+@pytest.mark.parametrize("chunks", [[1024] * 6, [4096, 2048]])
+def test_prepared_chunks_equal_the_plain_calls(chunks):
+    # the filter synthesised once (hyena_modal_prepare) and the chunks run
+    # without it give the bits of the plain calls and of the single pass
+    import torch
+    import hyena_long_convolution_b200 as hy
+    inp = make_modal_inputs(1, 6144, 520, 12, seed=41)
+    S0 = np.random.default_rng(41).standard_normal((1, 520, 12))
+    y1, s1 = check(inp, S0)
+    x = [to_dev_bf16(inp[k]) for k in ("x1", "x2", "x3")]
+    a, R, Ds = (to_dev_f32(inp[k]) for k in ("log_poles", "residues", "Dskip"))
+    ws = hy.ModalWorkspace(1, 520, 12)
+    S = to_dev_f32(S0)
+    y = torch.empty((1, 6144, 520), dtype=torch.bfloat16, device="cuda")
+    hy.modal_prepare(a, R, Ds, ws)
+    t0 = 0
+    for n in chunks:
+        hy.modal_long_conv_prepared(*(v[:, t0:t0 + n] for v in x), 12, ws, y=y[:, t0:t0 + n], state_in=S,
+                                    state_out=S)
+        t0 += n
+    hy.workspace_check(ws)
+    assert np.array_equal(bits_of(y), bits_of(y1))
+    assert np.array_equal(S.cpu().numpy(), s1.cpu().numpy())

@@ -104,3 +104,18 @@ def test_short_host_stream_is_bitwise_the_device_single_pass(B, L, D, K, chunk):
     if K == 128 and L == 5000:
         ref_y, ref_H = oracle.fir(inp["x1"], inp["x2"], inp["x3"], inp["taps"], inp["Dskip"], H0.astype(np.float64))
         assert_close(from_dev_bf16(yh.contiguous().view(torch.bfloat16)), ref_y, "host-buffer short conv")
+
+
+def test_host_stream_with_pageable_memory():
+    # pageable host buffers: the copies do not overlap, the result is the same
+    import torch
+    import hyena_long_convolution_b200 as hy
+    B, L, D, N = 1, 2000, 64, 8
+    inp = make_modal_inputs(B, L, D, N, seed=3)
+    a, R, Ds = (to_dev_f32(inp[k]) for k in ("log_poles", "residues", "Dskip"))
+    y_dev = hy.modal_long_conv(*(to_dev_bf16(inp[k]) for k in ("x1", "x2", "x3")), a, R, Ds)
+    xh = [torch.from_numpy(np.ascontiguousarray(inp[k]).view(np.int16)) for k in ("x1", "x2", "x3")]
+    yh = torch.zeros((B, L, D), dtype=torch.int16)
+    hy.modal_long_conv_host(*xh, a, R, Ds, y=yh, workspace=hy.HostWorkspace(B, D, N, chunk=512))
+    torch.cuda.synchronize()
+    assert torch.equal(yh, y_dev.view(torch.int16).cpu())

@@ -206,3 +206,28 @@ def test_prepared_chunks_equal_the_plain_calls(chunks):
     hy.workspace_check(ws)
     assert np.array_equal(bits_of(y), bits_of(y1))
     assert np.array_equal(S.cpu().numpy(), s1.cpu().numpy())
+
+
+@pytest.mark.parametrize("L", [1000, 5000])
+def test_degenerate_filters(L):
+    # p = 1 (a = 0: every mode a running sum), p underflowing to a denormal or
+    # zero (a = -100, -200: the filter is R at lag 0 only), R = 0 (y = D v),
+    # N = 1, and ordinary modes, channel block by channel block; the short
+    # path (L = 1000) and the look-back kernel (L = 5000) against the oracle,
+    # each channel against its own scale.
+    inp = make_modal_inputs(1, L, 64, 4, seed=L)
+    a = inp["log_poles"].copy()
+    R = inp["residues"].copy()
+    a[0:16] = 0.0
+    a[16:24] = -100.0
+    a[24:32] = -200.0
+    R[32:48] = 0.0
+    inp = dict(inp, log_poles=a, residues=R)
+    y, S = run_gpu(inp)
+    ref_y, ref_S = oracle.modal_recurrence(inp["x1"], inp["x2"], inp["x3"], a, R, inp["Dskip"])
+    assert_close(from_dev_bf16(y), ref_y, f"degenerate filters L={L}", per_channel=True)
+    rel, _ = metrics(S.cpu().numpy().astype(np.float64), ref_S)
+    assert rel <= STATE_TOL
+    # a single real mode
+    one = make_modal_inputs(2, L, 72, 1, seed=L + 1)
+    check(one, np.random.default_rng(L).standard_normal((2, 72, 1)), what=f"N=1 L={L}")

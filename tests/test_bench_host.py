@@ -1,6 +1,6 @@
 """The benchmark's roofline arithmetic and records, on the host (no GPU):
 algorithmic bytes and flops per channel-token as the design states them, the
-bound each workload is judged against, and the DRAM-traffic records, which
+bound each workload is measured against, and the DRAM-traffic records, which
 apply only while the kernel sources they were taken from are unchanged."""
 import json
 import os

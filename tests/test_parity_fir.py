@@ -82,6 +82,36 @@ def test_chunked_is_bitwise_single_pass(K, chunks):
     assert np.array_equal(Hc.cpu().numpy(), H1.cpu().numpy())
 
 
+@pytest.mark.parametrize("K", [33, 128])
+def test_ranges_of_many_tiles(K):
+    # 3 x 17 x 8 = 408 tiles of 64 channels x 128 tokens, more than a B200 has
+    # SMs: the long-filter kernel then walks ranges of several tiles that cross
+    # from one (batch row, channel group) sequence into the next, with ragged
+    # L and D, a carried window and both input layouts.
+    import torch
+    import hyena_long_convolution_b200 as hy
+    B, L, D = 3, 1000, 1032
+    inp = make_fir_inputs(B, L, D, K, seed=K + 11, with_skip=True)
+    H = np.random.default_rng(K).standard_normal((B, K - 1, D)).astype(np.float32).astype(np.float64)
+    y, Hout = check(inp, H)
+    # the interleaved per-channel triples give the same bits
+    xp = to_dev_bf16(np.stack([inp["x1"], inp["x2"], inp["x3"]], axis=3).reshape(B, L, 3 * D))
+    yt = hy.short_conv_packed(xp, 1, to_dev_bf16(inp["taps"]), to_dev_f32(inp["Dskip"]), hist_in=to_dev_f32(H))
+    torch.cuda.synchronize()
+    assert np.array_equal(bits_of(yt), bits_of(y))
+    # chunk boundaries move every range and tile; each output's sum does not change
+    xs = [to_dev_bf16(inp[k]) for k in ("x1", "x2", "x3")]
+    taps, Ds = to_dev_bf16(inp["taps"]), to_dev_f32(inp["Dskip"])
+    Hc = to_dev_f32(H)
+    parts = []
+    for t0, t1 in ((0, 500), (500, 1000)):
+        parts.append(hy.short_conv(*(x[:, t0:t1].contiguous() for x in xs), taps, Ds, hist_in=Hc, hist_out=Hc))
+    yc = torch.cat(parts, dim=1)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits_of(yc), bits_of(y))
+    assert np.array_equal(Hc.cpu().numpy(), Hout.cpu().numpy())
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("K", list(WORKLOAD_SHAPES["fir_8k"]["K"]))
 def test_fir_8k_full_size(K):

@@ -54,8 +54,11 @@ XSource packed_source(const hyena_bf16_t *xp, long long ld, int group)
 // chains): dims {group, D / group, L, B}, the group stride 3 group elements
 // (unused for a single group).  Triples: one map over the interleaved rows,
 // dims {3D, 1, L, B}, box of `rows` tokens x 3 width values (width channels'
-// triples).
-bool encode_x_map(CUtensorMap *m, const XSource &xs, int k, int B, int L, int D, int rows, int width = 64)
+// triples).  `promo`: how far L2 widens each row request; 256 bytes suits
+// grids whose concurrent CTAs read neighbouring channel groups (the widened
+// half is theirs), 128 bytes a persistent grid whose CTAs are far apart.
+bool encode_x_map(CUtensorMap *m, const XSource &xs, int k, int B, int L, int D, int rows, int width = 64,
+                  CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B)
 {
     std::call_once(g_encode_once, resolve_encode);
     if (g_encode == nullptr) return false;
@@ -89,8 +92,7 @@ bool encode_x_map(CUtensorMap *m, const XSource &xs, int k, int B, int L, int D,
     cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
     const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<hyena_bf16_t *>(xs.x[k]), dims,
                                 strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                                CU_TENSOR_MAP_SWIZZLE_NONE, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -238,10 +240,13 @@ hyena_status_t short_conv_impl(const XSource &xs, const hyena_bf16_t *taps, cons
     a.group = xs.group;
     a.hist_out = hist_out;
     CUtensorMap m1, m2, m3, h1, h2;
-    if (!encode_x_map(&m1, xs, 0, B, L, D, FT)) return HYENA_ERR_CUDA;
+    const CUtensorMapL2promotion promo =
+        fir_persistent(K) ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
+    if (!encode_x_map(&m1, xs, 0, B, L, D, FT, 64, promo)) return HYENA_ERR_CUDA;
     if (xs.triples) {
         m2 = m3 = m1;
-    } else if (!encode_x_map(&m2, xs, 1, B, L, D, FT) || !encode_x_map(&m3, xs, 2, B, L, D, FT)) {
+    } else if (!encode_x_map(&m2, xs, 1, B, L, D, FT, 64, promo) ||
+               !encode_x_map(&m3, xs, 2, B, L, D, FT, 64, promo)) {
         return HYENA_ERR_CUDA;
     }
     if (a.HR > 0) {

@@ -164,6 +164,10 @@ constexpr int FRW = FT / FW;  // output rows per warp
 
 inline int fir_halo_rows(int K) { return K <= 1 ? 0 : ((K - 1 + 7) / 8) * 8; }
 
+// Filters longer than 8 taps run the persistent kernel (one CTA per SM walking
+// tile ranges); shorter ones one CTA per tile.
+inline bool fir_persistent(int K) { return K > 8; }
+
 struct FirArgs {
     const uint16_t *taps;
     const float *Dskip;

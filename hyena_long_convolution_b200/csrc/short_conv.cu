@@ -458,6 +458,7 @@ __global__ void __launch_bounds__(FW * 32, 1)
 // output is the persistent kernel's (taps in lag order from a zero
 // accumulator).
 constexpr int kSmallMaxK = 8;
+static_assert(kSmallMaxK == 8, "fir_persistent() routes filters of more than 8 taps away");
 constexpr int kSmallHalf = 8;  // outputs per pass
 
 __host__ __device__ inline size_t fir_small_smem_bytes(int HR, int K, bool tri)
@@ -688,7 +689,7 @@ int launch_fir(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &
                       "fir: set max dynamic shared memory");
             configured_device = dev;
         }
-        if (a.K <= kSmallMaxK) {
+        if (!fir_persistent(a.K)) {
             const size_t smem = fir_small_smem_bytes(a.HR, a.K, triples);
             const dim3 grid((a.D + FCH - 1) / FCH, (a.L + FT - 1) / FT, a.B);
             if (triples)

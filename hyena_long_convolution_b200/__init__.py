@@ -44,6 +44,7 @@ __all__ = [
     "modal_state_init",
     "short_conv",
     "short_conv_packed",
+    "short_conv_dft",
     "short_decode",
     "short_decode_packed",
     "workspace_check",
@@ -390,6 +391,19 @@ def short_conv(x1, x2, x3, taps, Dskip=None, y=None, hist_in=None, hist_out=None
     taps: [D, K] bf16 in lag order (taps[c, k] multiplies v[t-k]);
     hist_in/hist_out: [B, K-1, D] fp32 or None (may be the same tensor).
     """
+    return _short_conv("hyena_short_conv", x1, x2, x3, taps, Dskip, y, hist_in, hist_out, stream)
+
+
+def short_conv_dft(x1, x2, x3, taps, Dskip=None, y=None, hist_in=None, hist_out=None, stream=None):
+    """short_conv computed on the tensor cores as overlap-save DFT-as-GEMM
+    (hyena_short_conv_dft): the same arguments; results agree with short_conv
+    to tf32 rounding.  The first call on a device copies the DFT tables with a
+    synchronous copy (make it before any CUDA graph capture).
+    """
+    return _short_conv("hyena_short_conv_dft", x1, x2, x3, taps, Dskip, y, hist_in, hist_out, stream)
+
+
+def _short_conv(entry, x1, x2, x3, taps, Dskip, y, hist_in, hist_out, stream):
     torch = _torch()
     s1, s2, s3 = _bld(x1, "x1"), _bld(x2, "x2"), _bld(x3, "x3")
     _same_ld(s1, s2, s3)
@@ -407,9 +421,9 @@ def short_conv(x1, x2, x3, taps, Dskip=None, y=None, hist_in=None, hist_out=None
     yB, yL, yD, ld_y = _bld(y, "y")
     if (yB, yL, yD) != (B, L, D):
         raise ValueError("y shape differs from x")
-    rc = lib().hyena_short_conv(_ptr(x1), _ptr(x2), _ptr(x3), ld, _ptr(taps), _ptr(Dskip), _ptr(y), ld_y,
-                                _ptr(hist_in), _ptr(hist_out), B, L, D, K, _stream(stream))
-    check("hyena_short_conv", rc)
+    rc = getattr(lib(), entry)(_ptr(x1), _ptr(x2), _ptr(x3), ld, _ptr(taps), _ptr(Dskip), _ptr(y), ld_y,
+                               _ptr(hist_in), _ptr(hist_out), B, L, D, K, _stream(stream))
+    check(entry, rc)
     return y
 
 

@@ -33,6 +33,7 @@ SIGNATURES = {
     "hyena_last_launch_count": (_I, []),
     "hyena_last_error_message": (ctypes.c_char_p, []),
     "hyena_short_conv": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I64, _P, _P, _I, _I, _I, _I, _P]),
+    "hyena_short_conv_dft": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I64, _P, _P, _I, _I, _I, _I, _P]),
     "hyena_modal_long_conv_workspace_size": (_SZ, [_I, _I, _I]),
     "hyena_modal_workspace_init": (_I, [_P, _SZ, _P]),
     "hyena_modal_long_conv": (_I, [_P, _P, _P, _I64, _P, _P, _P, _P, _I64, _P, _P,

@@ -202,9 +202,11 @@ using namespace hyena;
 
 namespace {
 
+// dft: the tensor-core DFT-as-GEMM kernel instead of the FP32 SIMT kernels
+// (separate or packed inputs only).
 hyena_status_t short_conv_impl(const XSource &xs, const hyena_bf16_t *taps, const float *Dskip, hyena_bf16_t *y,
                                int64_t ld_y, const float *hist_in, float *hist_out, int B, int L, int D, int K,
-                               void *stream)
+                               void *stream, bool dft = false)
 {
     hyena_status_t st = HYENA_OK;
     if (K < 1 || K > HYENA_MAX_TAPS) return K < 1 ? HYENA_ERR_INVALID_ARG : HYENA_ERR_UNSUPPORTED;
@@ -239,6 +241,17 @@ hyena_status_t short_conv_impl(const XSource &xs, const hyena_bf16_t *taps, cons
     a.ld_x = xs.ld;
     a.group = xs.group;
     a.hist_out = hist_out;
+    if (dft) {
+        if (xs.triples) return HYENA_ERR_UNSUPPORTED;
+        CUtensorMap m1, m2, m3;
+        if (!encode_x_map(&m1, xs, 0, B, L, D, FT) || !encode_x_map(&m2, xs, 1, B, L, D, FT) ||
+            !encode_x_map(&m3, xs, 2, B, L, D, FT))
+            return HYENA_ERR_CUDA;
+        const int n = launch_fir_dft(m1, m2, m3, a, s);
+        if (n < 0) return HYENA_ERR_CUDA;
+        g_last_launches = n;
+        return HYENA_OK;
+    }
     CUtensorMap m1, m2, m3, h1, h2;
     const CUtensorMapL2promotion promo =
         fir_persistent(K) ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
@@ -469,6 +482,17 @@ hyena_status_t hyena_short_conv(const hyena_bf16_t *x1, const hyena_bf16_t *x2, 
     if (st != HYENA_OK) return st;
     return short_conv_impl(separate_source(x1, x2, x3, ld_x, D), taps, Dskip, y, ld_y, hist_in, hist_out, B, L, D,
                            K, stream);
+}
+
+hyena_status_t hyena_short_conv_dft(const hyena_bf16_t *x1, const hyena_bf16_t *x2, const hyena_bf16_t *x3,
+                                    int64_t ld_x, const hyena_bf16_t *taps, const float *Dskip, hyena_bf16_t *y,
+                                    int64_t ld_y, const float *hist_in, float *hist_out, int B, int L, int D, int K,
+                                    void *stream)
+{
+    const hyena_status_t st = check_x(x1, x2, x3, ld_x, y, ld_y, B, L, D);
+    if (st != HYENA_OK) return st;
+    return short_conv_impl(separate_source(x1, x2, x3, ld_x, D), taps, Dskip, y, ld_y, hist_in, hist_out, B, L, D,
+                           K, stream, true);
 }
 
 hyena_status_t hyena_short_conv_packed(const hyena_bf16_t *xp, int64_t ld_x, int group, const hyena_bf16_t *taps,

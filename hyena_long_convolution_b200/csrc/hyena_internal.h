@@ -206,4 +206,13 @@ int launch_fir(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &
                const CUtensorMap &h1, const CUtensorMap &h2, const FirArgs &a,
                bool triples, cudaStream_t st);
 
+// hist_out (the last K-1 values of v), when requested: 0 or 1 launches, or -1.
+int launch_fir_history(const FirArgs &a, cudaStream_t st);
+
+// The FIR as overlap-save DFT-as-GEMM on the tensor cores (fir_dft.cu): tile
+// maps m1..m3 of FT rows over separate or packed inputs (no triples), then the
+// history as launch_fir_history.
+int launch_fir_dft(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &m3, const FirArgs &a,
+                   cudaStream_t st);
+
 }  // namespace hyena

@@ -711,19 +711,24 @@ int launch_fir(const CUtensorMap &m1, const CUtensorMap &m2, const CUtensorMap &
         HYENA_TRY(cudaGetLastError(), "fir launch");
         ++launches;
     }
-    if (a.hist_out != nullptr && a.K > 1) {
-        const int H = a.K - 1;
-        if (a.hist_in == a.hist_out && a.L > 0 && a.L < H) {
-            const int threads = a.B * (a.D / 2);
-            fir_history_kernel<<<(threads + 255) / 256, 256, 0, st>>>(a);
-        } else {
-            const long long threads = static_cast<long long>(a.B) * H * (a.D / 2);
-            fir_history_rows_kernel<<<static_cast<unsigned int>((threads + 255) / 256), 256, 0, st>>>(a);
-        }
-        HYENA_TRY(cudaGetLastError(), "fir history launch");
-        ++launches;
+    const int nh = launch_fir_history(a, st);
+    if (nh < 0) return -1;
+    return launches + nh;
+}
+
+int launch_fir_history(const FirArgs &a, cudaStream_t st)
+{
+    if (a.hist_out == nullptr || a.K <= 1) return 0;
+    const int H = a.K - 1;
+    if (a.hist_in == a.hist_out && a.L > 0 && a.L < H) {
+        const int threads = a.B * (a.D / 2);
+        fir_history_kernel<<<(threads + 255) / 256, 256, 0, st>>>(a);
+    } else {
+        const long long threads = static_cast<long long>(a.B) * H * (a.D / 2);
+        fir_history_rows_kernel<<<static_cast<unsigned int>((threads + 255) / 256), 256, 0, st>>>(a);
     }
-    return launches;
+    HYENA_TRY(cudaGetLastError(), "fir history launch");
+    return 1;
 }
 
 }  // namespace hyena

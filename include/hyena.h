@@ -98,6 +98,33 @@ hyena_status_t hyena_short_conv(const hyena_bf16_t *x1, const hyena_bf16_t *x2,
                                 int B, int L, int D, int K, void *stream);
 
 /*
+ * The same operator as hyena_short_conv, computed on the tensor cores as
+ * overlap-save DFT-as-GEMM: the FFT route of the Evo2-7B-262K model card,
+ * §Implementation Notes (hcl "via FFT", "Block dispatch" for the FIR
+ * cascades), restated as GEMMs with a shared real DFT matrix of 256 points
+ * so that channels are the MMA's N dimension (tcgen05 kind::tf32, fp32
+ * accumulation).  A second implementation for comparison with the FP32 SIMT
+ * kernels of hyena_short_conv; the arguments, layouts, ownership and error
+ * behaviour are those of hyena_short_conv.  Differences:
+ *  - v, the DFT matrices and the spectrum product are rounded to tf32 (11
+ *    significant bits) before each product; results agree with
+ *    hyena_short_conv to that rounding, not bit for bit;
+ *  - each output depends on where its 128-token block starts, so feeding a
+ *    sequence in chunks reproduces the single pass to rounding, not bit for
+ *    bit (use hyena_short_conv where chunked results must match exactly);
+ *  - hist_in values are rounded to tf32 like v (v = x1 x2 of bf16 inputs
+ *    is exact only in fp32).
+ * The first call on a device copies the DFT tables (384 KB of the library's
+ * device memory) with a synchronous copy: make it before any stream capture.
+ */
+hyena_status_t hyena_short_conv_dft(const hyena_bf16_t *x1, const hyena_bf16_t *x2,
+                                    const hyena_bf16_t *x3, int64_t ld_x,
+                                    const hyena_bf16_t *taps, const float *Dskip,
+                                    hyena_bf16_t *y, int64_t ld_y,
+                                    const float *hist_in, float *hist_out,
+                                    int B, int L, int D, int K, void *stream);
+
+/*
  * Bytes of device workspace hyena_modal_long_conv needs for B, D, N
  * (independent of L).  Returns 0 for invalid sizes.
  */

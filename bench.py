@@ -49,6 +49,9 @@ WORKLOADS = {
                  desc="hcs explicit FIR K=7, B=2 L=8192 D=4096"),
     "fir128": dict(kind="fir", B=2, L=8192, D=4096, K=128, seed=1,
                    desc="hcm explicit FIR K=128, B=2 L=8192 D=4096"),
+    # the same operator as overlap-save DFT-as-GEMM on the tensor cores (tf32)
+    "fir128_dft": dict(kind="fir", B=2, L=8192, D=4096, K=128, seed=1, dft=True,
+                       desc="hcm explicit FIR K=128, B=2 L=8192 D=4096, tensor-core DFT-as-GEMM (tf32)"),
     # inputs read from one projection buffer interleaved per channel triple
     # (x1_c, x2_c, x3_c adjacent), the in_proj output layout
     "modal32k_triples": dict(kind="modal", B=1, L=32768, D=4096, N=16, seed=2, chunk=None, group=1,
@@ -106,6 +109,26 @@ def algorithmic_bytes(wl):
     return per_call * wl["L"]
 
 
+# Tensor-core work of the DFT-as-GEMM FIR per channel-token: per 64 channels x
+# 128 outputs, the taps' spectrum (2 x 128 x 64 x 128 MACs), the window's
+# (2 x 128 x 64 x 256) and the inverse (128 x 64 x 256): 1024 MACs.
+DFT_FLOPS_PER_CHTOK = 2 * 1024
+# Nominal dense tf32 / bf16 tensor rates of a B200 (1.1 and 2.25 PFLOP/s).
+TF32_PER_BF16 = 1.1 / 2.25
+
+
+def tensor_peak_tflops_tf32():
+    """Dense tf32 tensor peak: the measured bf16 GEMM rate (burst) when the
+    measured-peaks file is present, else a fallback of 1590 TFLOP/s (an
+    earlier cuBLAS bf16 measurement on a B200), times the nominal tf32 / bf16
+    ratio."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]) * TF32_PER_BF16, "measured bf16_tflops x nominal tf32/bf16"
+    except Exception:
+        return 1590.0 * TF32_PER_BF16, "fallback bf16 1590 TFLOP/s x nominal tf32/bf16"
+
+
 def flops_per_chtok(wl):
     """Algorithmic flops per channel-token: the recurrence form's 2N FMAs
     (hcl; complex modes: 6N, four for p s + v and two for Re(R s)) or K FMAs
@@ -124,6 +147,8 @@ def kernel_fma_per_chtok(wl):
     gate and the skip."""
     if wl["kind"] == "modal":
         return (10 * wl["N"] if wl.get("cx") else 3 * wl["N"]) + 4
+    if wl.get("dft"):
+        return None  # the arithmetic is on the tensor cores
     return wl["K"] + 3
 
 
@@ -146,6 +171,9 @@ KERNEL_SOURCES = {
     "fir": ("hyena_long_convolution_b200/csrc/short_conv.cu",
             "hyena_long_convolution_b200/csrc/hyena_device.cuh",
             "hyena_long_convolution_b200/csrc/hyena_internal.h"),
+    "fir_dft": ("hyena_long_convolution_b200/csrc/fir_dft.cu",
+                "hyena_long_convolution_b200/csrc/hyena_device.cuh",
+                "hyena_long_convolution_b200/csrc/hyena_internal.h"),
 }
 
 
@@ -168,7 +196,9 @@ def recorded_traffic(workload):
             rec = json.load(f).get(workload)
     except Exception:
         return None
-    if not rec or rec.get("kernel_sources_sha256_16") != kernel_source_hash(WORKLOADS[workload]["kind"]):
+    wl = WORKLOADS[workload]
+    kind = "fir_dft" if wl.get("dft") else wl["kind"]
+    if not rec or rec.get("kernel_sources_sha256_16") != kernel_source_hash(kind):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -499,7 +529,8 @@ class Step:
                                    state_out=self.S, workspace=self.ws)
                 n += hy.last_launch_count()
         else:
-            hy.short_conv(d["x1"], d["x2"], d["x3"], d["taps"], None, y=self.y)
+            conv = hy.short_conv_dft if wl.get("dft") else hy.short_conv
+            conv(d["x1"], d["x2"], d["x3"], d["taps"], None, y=self.y)
             n += hy.last_launch_count()
         self.launches = n
 
@@ -551,7 +582,7 @@ def e2e_leg(wl, host, dev, device, steps, warmup):
     # Prefill with separate inputs (real modes, FIR) streams its host buffers
     # through the library's host-buffer entry points (chunks, copies in both
     # directions overlapping the computation); everything else copies here.
-    streamed = not (wl.get("cx") or wl.get("group") or wl.get("decode"))
+    streamed = not (wl.get("cx") or wl.get("group") or wl.get("decode") or wl.get("dft"))
     on_host = ("x1", "x2", "x3") if streamed else ()
     dx = {k: torch.empty(v.shape, dtype=v.dtype, device=device) for k, v in hx.items() if k not in on_host}
     y_host = torch.empty((wl["B"], wl["L"], wl["D"]), dtype=torch.int16).pin_memory()
@@ -601,7 +632,8 @@ def e2e_leg(wl, host, dev, device, steps, warmup):
         elif wl["kind"] == "modal":
             hy.modal_long_conv(bf["x1"], bf["x2"], bf["x3"], dx["a"], dx["R"], dx["Ds"], y=y, workspace=ws)
         else:
-            hy.short_conv(bf["x1"], bf["x2"], bf["x3"], dx["taps"].view(torch.bfloat16), None, y=y)
+            conv = hy.short_conv_dft if wl.get("dft") else hy.short_conv
+            conv(bf["x1"], bf["x2"], bf["x3"], dx["taps"].view(torch.bfloat16), None, y=y)
         y_host.copy_(y.view(torch.int16), non_blocking=True)
 
     per = time_steps(step, steps, warmup, device)
@@ -667,7 +699,13 @@ def run_gpu(args, wl):
     # the algorithmic flops take longer at the SIMT peak (long explicit FIRs).
     alu_peak = alu_peak_tflops()
     flops = flops_per_chtok(wl) * chtok
-    if flops / (alu_peak * 1e12) > step_bytes / (peak * 1e9):
+    if wl.get("dft"):
+        # the DFT path's own arithmetic on the tensor cores bounds it
+        tc_peak, tc_src = tensor_peak_tflops_tf32()
+        mma_flops = DFT_FLOPS_PER_CHTOK * chtok
+        roof = {"bound": "tensor", "achieved": mma_flops / (avg_ms / 1e3) / 1e12, "peak": tc_peak,
+                "unit": "TFLOP/s", "peak_source": tc_src, "algorithmic_flops_per_launch": mma_flops}
+    elif flops / (alu_peak * 1e12) > step_bytes / (peak * 1e9):
         roof = {"bound": "alu", "achieved": flops / (avg_ms / 1e3) / 1e12, "peak": alu_peak, "unit": "TFLOP/s",
                 "peak_source": "derived: SMs x 128 FP32 lanes x 2 flops x max SM clock",
                 "algorithmic_flops_per_launch": flops}
@@ -677,7 +715,8 @@ def run_gpu(args, wl):
     roof["frac"] = roof["achieved"] / roof["peak"]
     # The kernels' own arithmetic floor: their FMA-pipe work at the SIMT peak
     # (a step cannot beat it however well its memory traffic is hidden).
-    fma_floor_ms = kernel_fma_per_chtok(wl) * chtok / (alu_peak * 1e12 / 2) * 1e3 if not wl.get("decode") else None
+    fma_pc = kernel_fma_per_chtok(wl)
+    fma_floor_ms = fma_pc * chtok / (alu_peak * 1e12 / 2) * 1e3 if fma_pc and not wl.get("decode") else None
     roof.update({"traffic": traffic, "algorithmic_bytes_per_step": step_bytes,
                  "hbm_frac": achieved / peak, "kernel_ms_min": per_sorted[0], "kernel_ms_avg": avg_ms,
                  "fma_floor_ms": fma_floor_ms,

@@ -69,13 +69,13 @@ def modal(lib, **kw):
                                      args["ws"], args["ws_bytes"], args["st"])
 
 
-def fir(lib, **kw):
+def fir(lib, entry="hyena_short_conv", **kw):
     args = dict(x1=A, x2=A, x3=A, ld_x=64, taps=A, ds=None, y=A + 4096, ld_y=64, h_in=None,
                 h_out=None, B=1, L=16, D=64, K=7, st=None)
     args.update(kw)
-    return lib.hyena_short_conv(args["x1"], args["x2"], args["x3"], args["ld_x"], args["taps"],
-                                args["ds"], args["y"], args["ld_y"], args["h_in"], args["h_out"],
-                                args["B"], args["L"], args["D"], args["K"], args["st"])
+    return getattr(lib, entry)(args["x1"], args["x2"], args["x3"], args["ld_x"], args["taps"],
+                               args["ds"], args["y"], args["ld_y"], args["h_in"], args["h_out"],
+                               args["B"], args["L"], args["D"], args["K"], args["st"])
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -96,8 +96,10 @@ def test_modal_rejects_bad_arguments(kw, code):
     (dict(K=0), INVALID), (dict(K=129), UNSUP), (dict(ld_x=8), INVALID), (dict(x1=A + 6), ALIGN),
     (dict(taps=A + 2), ALIGN), (dict(h_in=A + 4), ALIGN), (dict(D=12, ld_x=16, ld_y=16), ALIGN),
 ])
-def test_short_conv_rejects_bad_arguments(kw, code):
-    assert fir(hy.lib(), **kw) == code
+@pytest.mark.parametrize("entry", ["hyena_short_conv", "hyena_short_conv_dft"])
+def test_short_conv_rejects_bad_arguments(kw, code, entry):
+    # the tensor-core FIR takes the same arguments and refuses the same ones
+    assert fir(hy.lib(), entry, **kw) == code
 
 
 def mdec(lib, x1=A, x2=A, x3=A, ld_x=64, a=A, R=A, Ds=None, y=A, ld_y=64, state=A, B=1, D=64, N=8):

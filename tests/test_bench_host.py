@@ -65,3 +65,31 @@ def test_traffic_records_follow_the_kernel_sources(tmp_path, monkeypatch):
     assert bench.recorded_traffic("modal32k") is None
     monkeypatch.setattr(bench, "kernel_source_hash", lambda kind="modal": "0000000000000000")
     assert bench.recorded_traffic("modal32k") == 1
+
+
+def test_tensor_core_fir_line():
+    # the DFT-as-GEMM FIR: its method's tf32 MMA work per channel-token (the
+    # two spectra and the inverse per 64 channels x 128 outputs), no SIMT FMA
+    # floor, and a tf32 peak of the bf16 figure times the nominal ratio
+    wl = bench.WORKLOADS["fir128_dft"]
+    macs = 2 * 128 * 64 * 128 + 2 * 128 * 64 * 256 + 128 * 64 * 256
+    assert bench.DFT_FLOPS_PER_CHTOK == 2 * macs // (64 * 128)
+    assert bench.kernel_fma_per_chtok(wl) is None
+    assert bench.algorithmic_bytes(wl) == bench.algorithmic_bytes(bench.WORKLOADS["fir128"])
+    peak, src = bench.tensor_peak_tflops_tf32()
+    assert peak > 0 and "tf32/bf16" in src
+    assert abs(bench.TF32_PER_BF16 - 1.1 / 2.25) < 1e-12
+
+
+def test_tensor_core_fir_traffic_follows_its_own_sources(tmp_path, monkeypatch):
+    # the DFT path's record is keyed by the hash of fir_dft.cu and the shared
+    # headers, not by the SIMT FIR's
+    fake = tmp_path / "profiles"
+    fake.mkdir()
+    (fake / "traffic.json").write_text(json.dumps(
+        {"fir128_dft": {"dram_bytes_per_launch": 7, "kernel_sources_sha256_16": "abc"}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda kind="modal": "abc" if kind == "fir_dft" else "zzz")
+    assert bench.recorded_traffic("fir128_dft") == 7
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda kind="modal": "abc" if kind == "fir" else "zzz")
+    assert bench.recorded_traffic("fir128_dft") is None

@@ -104,3 +104,25 @@ def test_fir128_full_size():
     y, _ = run_dft(inp)
     ref, _ = oracle.fir(inp["x1"], inp["x2"], inp["x3"], inp["taps"], None, None)
     assert_close(from_dev_bf16(y), ref, "dft FIR 8K K=128")
+
+
+def test_row_strides_and_aliased_window():
+    # x1, x2, x3 as three views of one [B, L, 3D + pad] buffer (row stride >
+    # D), y with a padded row stride, and hist_in == hist_out
+    import torch
+    import hyena_long_convolution_b200 as hy
+    B, L, D, K = 2, 700, 192, 128
+    inp = make_fir_inputs(B, L, D, K, seed=33, with_skip=True)
+    H0 = np.random.default_rng(5).standard_normal((B, K - 1, D)).astype(np.float32)
+    wide = np.concatenate([inp["x1"], inp["x2"], inp["x3"], np.zeros((B, L, 64), np.uint16)], axis=2)
+    buf = to_dev_bf16(wide)
+    xs = [buf[..., :D], buf[..., D:2 * D], buf[..., 2 * D:3 * D]]
+    ybuf = torch.zeros((B, L, D + 32), dtype=torch.bfloat16, device="cuda")
+    y = ybuf[..., :D]
+    H = torch.from_numpy(H0).cuda()
+    hy.short_conv_dft(*xs, to_dev_bf16(inp["taps"]), to_dev_f32(inp["Dskip"]), y=y, hist_in=H, hist_out=H)
+    torch.cuda.synchronize()
+    ref_y, ref_H = oracle.fir(inp["x1"], inp["x2"], inp["x3"], inp["taps"], inp["Dskip"], H0.astype(np.float64))
+    assert_close(from_dev_bf16(y), ref_y, "dft fir, strided views")
+    assert np.array_equal(H.cpu().numpy().astype(np.float64), ref_H)
+    assert torch.count_nonzero(ybuf[..., D:]) == 0  # the padding columns are not written

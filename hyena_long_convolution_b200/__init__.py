@@ -64,6 +64,11 @@ def _torch():
 def _stream(stream):
     torch = _torch()
     if stream is None:
+        # the current stream of the current device; torch's raw query skips
+        # building a Stream object (3.5 us of a ~19 us decode call)
+        raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+        if raw is not None:
+            return ctypes.c_void_p(raw(torch.cuda.current_device()))
         return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     if isinstance(stream, torch.cuda.Stream):
         return ctypes.c_void_p(stream.cuda_stream)

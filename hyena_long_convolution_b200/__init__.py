@@ -68,15 +68,17 @@ def _stream(stream):
         # building a Stream object (3.5 us of a ~19 us decode call)
         raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
         if raw is not None:
-            return ctypes.c_void_p(raw(torch.cuda.current_device()))
-        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+            return raw(torch.cuda.current_device())
+        return torch.cuda.current_stream().cuda_stream
     if isinstance(stream, torch.cuda.Stream):
-        return ctypes.c_void_p(stream.cuda_stream)
-    return ctypes.c_void_p(int(stream))
+        return stream.cuda_stream
+    return int(stream)
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    # a plain integer: ctypes converts it through the entry point's c_void_p
+    # argument type (None is NULL)
+    return None if t is None else t.data_ptr()
 
 
 def _bld(x, name):
@@ -330,11 +332,13 @@ def _bd(x, name):
     """One token per batch row: [B, D] or [B, 1, D] bf16 with unit channel
     stride -> (B, D, ld), element (b, c) at b * ld + c."""
     torch = _torch()
-    if x.dtype != torch.bfloat16 or not x.is_cuda or x.dim() not in (2, 3) or (x.dim() == 3 and x.shape[1] != 1):
+    sh = x.shape  # one query each of shape and strides: this runs once per tensor per token
+    if x.dtype is not torch.bfloat16 or not x.is_cuda or len(sh) not in (2, 3) or (len(sh) == 3 and sh[1] != 1):
         raise ValueError(f"{name} must be a bf16 CUDA tensor [B, D] or [B, 1, D]")
-    if x.stride(-1) != 1:
+    st = x.stride()
+    if st[-1] != 1:
         raise ValueError(f"{name} must have unit channel stride")
-    return x.shape[0], x.shape[-1], x.stride(0)
+    return sh[0], sh[-1], st[0]
 
 
 def modal_decode(x1, x2, x3, log_poles, residues, Dskip, state, y=None, stream=None):
